@@ -1,0 +1,786 @@
+// kvq_decode.cu -- split-K paged GQA decode attention over the quantized cache.
+//
+// What it computes (one query token per sequence, query head h reading kv-head
+// h / G): out = softmax(scale * q K^T) V over the sequence's tokens, with K and
+// V taken from the cache as code x scale.  "NInfer KV Cache 量化指南" (why quantise:
+// every decoded token re-reads the whole KV, so stored bytes set decode speed)
+// and "FP8 KV Cache如何提速 ... 长上下文推理" (the bottleneck is memory bandwidth,
+// not arithmetic) make this a streaming kernel: its roofline is HBM bandwidth.
+//
+// Design (B200, sm_100a):
+//  * Persistent CTAs (4 warps).  The page-heads of the whole batch, ordered
+//    (sequence, kv-head, 8-head block, page), are cut into gridDim.x contiguous
+//    equal ranges, so ragged batches balance to within one page.
+//  * Each page slab (K codes, K scales, V codes, V scales of one kv-head: one
+//    contiguous range in HBM) arrives with ONE cp.async.bulk into a shared-memory
+//    stage, completion tracked by an mbarrier; `stages` slabs are in flight.
+//  * Warp w takes 16-token tiles w, w+4, ... of each page.  Codes are turned
+//    into fp16 (exact for every format) in registers straight from shared
+//    memory and fed to mma.sync m16n8k16 with the GQA group (<= 8 query heads)
+//    as N: S^T = K q^T with tokens as M, then O^T += V^T P^T with head_dim as M
+//    (movmatrix transposes the V and P fragments).  Group scales are folded
+//    into fp32 S (K) or into P (V); NVFP4 scales go into the operand, where
+//    code x scale is exact in fp16.  q is split into hi + lo halves so the
+//    scores keep ~22 bits.
+//  * Online softmax in the log2 domain per warp; the four warps merge in
+//    shared memory at the end of each (sequence, kv-head) segment.  A segment
+//    cut by a CTA range boundary writes a partial (max, sum, unnormalised
+//    output) and the last CTA to finish that segment merges all partials
+//    (arrival counter in the workspace, reset by the merger): no second launch.
+//  * Rotated K: q is rotated by the same normalised Hadamard-256 (orthonormal,
+//    so q.k is unchanged).  Rotated V: the output is rotated back (the matrix
+//    is symmetric and its own inverse).
+#include "kvq_internal.h"
+
+namespace kvq {
+
+constexpr int kDecThreads = 128;
+constexpr int kMaxStages = 8;
+constexpr int kMaxBatch = 4096;
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ------------------------------------------------------------ PTX helpers
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t phase) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(phase)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait: gives up after ~2^22 polls (each poll may suspend briefly).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t phase) {
+    for (int i = 0; i < (1 << 22); i++)
+        if (mbar_try_wait(bar, phase)) return true;
+    return false;
+}
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(src), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mma_f16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t movtrans(uint32_t x) {
+    uint32_t r;
+    asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(r) : "r"(x));
+    return r;
+}
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+__device__ __forceinline__ uint32_t f16_splat(uint32_t h16) { return (h16 & 0xFFFFu) * 0x10001u; }
+
+template <int NB>
+struct Bytes;   // NB bytes loaded from shared memory as 32-bit words
+template <>
+struct Bytes<8> { uint32_t w[2]; };
+template <>
+struct Bytes<16> { uint32_t w[4]; };
+template <>
+struct Bytes<32> { uint32_t w[8]; };
+
+// Load NB (8/16/32) logical bytes at logical offset `lb` of a code row whose
+// 16-byte chunks are permuted by `swz`.
+template <int NB>
+__device__ __forceinline__ Bytes<NB> lds_row(const uint8_t* row, int lb, int swz) {
+    Bytes<NB> b;
+    if constexpr (NB == 8) {
+        uint2 v = *reinterpret_cast<const uint2*>(row + phys_byte(lb, swz));
+        b.w[0] = v.x; b.w[1] = v.y;
+    } else if constexpr (NB == 16) {
+        uint4 v = *reinterpret_cast<const uint4*>(row + phys_byte(lb, swz));
+        b.w[0] = v.x; b.w[1] = v.y; b.w[2] = v.z; b.w[3] = v.w;
+    } else {
+        uint4 v0 = *reinterpret_cast<const uint4*>(row + phys_byte(lb, swz));
+        uint4 v1 = *reinterpret_cast<const uint4*>(row + phys_byte(lb + 16, swz));
+        b.w[0] = v0.x; b.w[1] = v0.y; b.w[2] = v0.z; b.w[3] = v0.w;
+        b.w[4] = v1.x; b.w[5] = v1.y; b.w[6] = v1.z; b.w[7] = v1.w;
+    }
+    return b;
+}
+
+// Four consecutive codes e0..e3 of one row (element `4 * step` of a lane's
+// slice) -> f16x2 pairs (e0,e1) and (e2,e3), without any scale.
+template <int KIND, int NB>
+__device__ __forceinline__ void codes4_f16(const Bytes<NB>& b, int step, uint32_t& x01, uint32_t& x23) {
+    if constexpr (kind_bits(KIND) == 16) {
+        x01 = b.w[2 * step];
+        x23 = b.w[2 * step + 1];
+    } else if constexpr (kind_bits(KIND) == 4) {
+        uint32_t h = (b.w[step >> 1] >> ((step & 1) * 16)) & 0xFFFFu;
+        x01 = dec_e2m1x2_f16x2(h & 0xFFu);
+        x23 = dec_e2m1x2_f16x2(h >> 8);
+    } else if constexpr (KIND == RK_INT8_G64) {
+        dec_int8x4_f16x2(b.w[step], x01, x23);
+    } else {
+        x01 = dec_e4m3x2_f16x2(b.w[step] & 0xFFFFu);
+        x23 = dec_e4m3x2_f16x2(b.w[step] >> 16);
+    }
+}
+
+template <int KK, int KV, int D>
+struct DecTraits {
+    static constexpr int KBITS = kind_bits(KK), VBITS = kind_bits(KV);
+    static constexpr int KCH = (KK == RK_E4M3_MX32) ? 2 : 4;   // k-steps per K load
+    static constexpr int VCH = (KV == RK_E4M3_MX32) ? 2 : 4;   // d-tiles per V load
+    static constexpr int KSTEPS = D / 16, DTILES = D / 16;
+    static constexpr int KCW = 16 * KCH, VCW = 16 * VCH;       // chunk widths in head_dim
+    static constexpr int KNB = 4 * KCH * KBITS / 8;            // bytes per lane per K row load
+    static constexpr int VNB = 4 * VCH * VBITS / 8;
+    static constexpr int EPL = D / 32;
+};
+
+// Cursor over this CTA's page-heads: (sequence b, head pair hh = h*HB + hb, page).
+struct Cursor {
+    int b, hh, page, npages;
+};
+
+__device__ __forceinline__ void cursor_next(Cursor& c, const int* pref, int B, int HH) {
+    if (++c.page < c.npages) return;
+    c.page = 0;
+    if (++c.hh < HH) return;
+    c.hh = 0;
+    do {
+        c.b++;
+    } while (c.b < B && pref[c.b + 1] == pref[c.b]);
+    c.npages = (c.b < B) ? pref[c.b + 1] - pref[c.b] : 0;
+}
+
+__device__ __forceinline__ void cursor_locate(Cursor& c, int64_t w, const int* pref, int B, int HH) {
+    int lo = 0, hi = B - 1;   // largest b with pref[b]*HH <= w
+    while (lo < hi) {
+        int mid = (lo + hi + 1) >> 1;
+        if ((int64_t)pref[mid] * HH <= w) lo = mid;
+        else hi = mid - 1;
+    }
+    while (lo < B - 1 && pref[lo + 1] == pref[lo]) lo++;   // skip empty sequences
+    c.b = lo;
+    c.npages = pref[lo + 1] - pref[lo];
+    int64_t idx = w - (int64_t)pref[lo] * HH;
+    c.hh = (int)(idx / c.npages);
+    c.page = (int)(idx % c.npages);
+}
+
+// CTA owning page-head w when W page-heads are cut into G equal ranges.
+__device__ __forceinline__ int owner_of(int64_t w, int64_t W, int G) {
+    return (int)(((w + 1) * G + W - 1) / W) - 1;
+}
+
+template <int KK, int KV, int D>
+__global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const DecodeParams p) {
+    using T = DecTraits<KK, KV, D>;
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int r = lane >> 2, j = lane & 3;
+    const int H = p.L.H, P = p.L.P, HB = p.HB, HH = H * HB, B = p.B;
+    const int64_t slab = p.L.slab;
+    const int NS = p.stages;
+
+    // shared memory carve-up
+    size_t off = ((size_t)NS * slab + 127) & ~(size_t)127;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + off);
+    off += 8 * kMaxStages;
+    float* osm = reinterpret_cast<float*>(smem + off);   // [8][D]: q staging / output combine
+    off += 8 * D * 4;
+    float* wml = reinterpret_cast<float*>(smem + off);   // [4 warps][m 8, l 8]
+    off += 4 * 16 * 4;
+    float* fin = reinterpret_cast<float*>(smem + off);   // [m 8][l 8] of the merged segment
+    off += 16 * 4;
+    int* flags = reinterpret_cast<int*>(smem + off);     // [0] abort, [1] last arriver
+    off += 16;
+    int* pref = reinterpret_cast<int*>(smem + off);      // [B + 1] page prefix
+
+    // ---- page prefix over the batch (block scan)
+    {
+        const int per = (B + kDecThreads - 1) / kDecThreads;
+        const int b0 = tid * per, b1 = min(B, b0 + per);
+        int local = 0;
+        for (int b = b0; b < b1; b++) {
+            int L = p.seq_lens[b];
+            int np = L > 0 ? (L + P - 1) / P : 0;
+            if (np > p.max_pages) {
+                np = p.max_pages;
+                atomicOr(p.status, kStatusBadPage);
+            }
+            local += np;
+        }
+        int incl = local;
+#pragma unroll
+        for (int m = 1; m < 32; m <<= 1) {
+            int v = __shfl_up_sync(0xffffffffu, incl, m);
+            if (lane >= m) incl += v;
+        }
+        if (lane == 31) wml[warp] = __int_as_float(incl);
+        if (tid == 0) {
+            flags[0] = 0;
+            flags[1] = 0;
+        }
+        __syncthreads();
+        int base = 0;
+        for (int w = 0; w < warp; w++) base += __float_as_int(wml[w]);
+        int run = base + incl - local;
+        for (int b = b0; b < b1; b++) {
+            pref[b] = run;
+            int L = p.seq_lens[b];
+            int np = L > 0 ? (L + P - 1) / P : 0;
+            run += min(np, p.max_pages);
+        }
+        if (tid == kDecThreads - 1) pref[B] = run;
+        if (B == 0 && tid == 0) pref[0] = 0;
+        __syncthreads();
+    }
+
+    // zero rows for empty sequences (one CTA per sequence)
+    for (int b = blockIdx.x; b < B; b += gridDim.x) {
+        if (pref[b + 1] == pref[b]) {
+            for (int i = tid; i < p.Hq * D; i += kDecThreads) {
+                int64_t o = (int64_t)b * p.Hq * D + i;
+                if (p.out_fp32) reinterpret_cast<float*>(p.out)[o] = 0.f;
+                else reinterpret_cast<__nv_bfloat16*>(p.out)[o] = __float2bfloat16_rn(0.f);
+            }
+        }
+    }
+
+    const int64_t W = (int64_t)pref[B] * HH;
+    if (W == 0) return;
+    const int G = (int)(((int64_t)gridDim.x < W) ? (int64_t)gridDim.x : W);
+    if ((int)blockIdx.x >= G) return;
+    const int64_t w0 = (int64_t)blockIdx.x * W / G, w1 = (int64_t)(blockIdx.x + 1) * W / G;
+    const int n = (int)(w1 - w0);
+
+    if (tid == 0) {
+        for (int s = 0; s < NS; s++) mbar_init(smem_u32(&bars[s]), 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+
+    // ---- producer: thread 0 keeps NS slabs in flight
+    Cursor pc{0, 0, 0, 0};
+    int issued = 0;
+    auto issue = [&](int s) {
+        int pid = p.block_table[(int64_t)pc.b * p.max_pages + pc.page];
+        if (pid < 0 || pid >= p.L.num_pages) {
+            atomicOr(p.status, kStatusBadPage);
+            pid = 0;
+        }
+        const uint8_t* src = p.slabs + ((int64_t)pid * H + pc.hh / HB) * slab;
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        uint32_t bar = smem_u32(&bars[s]);
+        mbar_expect_tx(bar, (uint32_t)slab);
+        bulk_g2s(smem_u32(smem + (size_t)s * slab), src, (uint32_t)slab, bar);
+    };
+    if (tid == 0) {
+        cursor_locate(pc, w0, pref, B, HH);
+        for (int s = 0; s < NS && issued < n; s++) {
+            issue(s);
+            cursor_next(pc, pref, B, HH);
+            issued++;
+        }
+    }
+
+    // ---- consumer state
+    Cursor cc;
+    cursor_locate(cc, w0, pref, B, HH);
+    uint32_t qh[T::KSTEPS][2], ql[T::KSTEPS][2];
+    float o[T::DTILES][4];
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+    bool seg_first = true;     // segment began at this CTA's first page
+
+    int i_stop = n;
+    for (int i = 0; i < n; i++) {
+        const int s = i % NS;
+        const bool seg_begin = (i == 0) || (cc.page == 0);
+        const int b = cc.b, h = cc.hh / HB, hb = cc.hh % HB;
+        if (seg_begin) {
+            seg_first = (i == 0);
+            // q rows of this 8-head block -> rotated, scaled fp32 in osm -> fragments
+#pragma unroll
+            for (int k = 0; k < 2; k++) {
+                const int nh = warp + 4 * k;
+                const int gq = hb * 8 + nh;
+                float x[8];
+                if (gq < p.G) {
+                    const uint16_t* qrow = p.q + ((int64_t)b * p.Hq + h * p.G + gq) * D + lane * T::EPL;
+#pragma unroll
+                    for (int e = 0; e < T::EPL; e++) x[e] = bf16_bits_to_f32(qrow[e]);
+                    if constexpr (D == 256) {
+                        if (p.rot_k) fwht256_warp(x, lane);
+                    }
+#pragma unroll
+                    for (int e = 0; e < T::EPL; e++) x[e] *= p.q_mult;
+                } else {
+#pragma unroll
+                    for (int e = 0; e < T::EPL; e++) x[e] = 0.f;
+                }
+#pragma unroll
+                for (int e = 0; e < T::EPL; e++) osm[nh * D + lane * T::EPL + e] = x[e];
+            }
+            __syncthreads();
+#pragma unroll
+            for (int st = 0; st < T::KSTEPS; st++) {
+                const int c = st / T::KCH, ks = st % T::KCH;
+                const int d0 = T::KCW * c + 4 * T::KCH * j + 4 * ks;
+                const float* qr = osm + r * D + d0;
+                float v[4] = {qr[0], qr[1], qr[2], qr[3]};
+                float lo[4];
+                if constexpr (KK == RK_BF16RAW) {
+#pragma unroll
+                    for (int e = 0; e < 4; e++) lo[e] = v[e] - __bfloat162float(__float2bfloat16_rn(v[e]));
+                    qh[st][0] = pack_bf16(v[0], v[1]);
+                    qh[st][1] = pack_bf16(v[2], v[3]);
+                    ql[st][0] = pack_bf16(lo[0], lo[1]);
+                    ql[st][1] = pack_bf16(lo[2], lo[3]);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 4; e++) lo[e] = v[e] - __half2float(__float2half_rn(v[e]));
+                    qh[st][0] = pack_f16(v[0], v[1]);
+                    qh[st][1] = pack_f16(v[2], v[3]);
+                    ql[st][0] = pack_f16(lo[0], lo[1]);
+                    ql[st][1] = pack_f16(lo[2], lo[3]);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < T::DTILES; u++) o[u][0] = o[u][1] = o[u][2] = o[u][3] = 0.f;
+            m0 = m1 = -INFINITY;
+            l0 = l1 = 0.f;
+        }
+
+        // wait for the slab
+        if (!mbar_wait(smem_u32(&bars[s]), (uint32_t)((i / NS) & 1))) {
+            atomicOr(p.status, kStatusWaitTimeout);
+            flags[0] = 1;
+        }
+
+        // ---- compute: 16-token tiles of this page
+        const uint8_t* stg = smem + (size_t)s * slab;
+        const uint8_t* kcodes = stg;
+        const uint8_t* kscl = stg + p.L.off_ks;
+        const uint8_t* vcodes = stg + p.L.off_vc;
+        const uint8_t* vscl = stg + p.L.off_vs;
+        const int seq_len = p.seq_lens[b];
+        for (int mt = warp; mt < P / 16; mt += 4) {
+            const int valid = seq_len - (cc.page * P + mt * 16);
+            if (valid <= 0) break;
+            const int ta = mt * 16 + r, tb = ta + 8;
+            // ---------- S^T = K q^T
+            float sc[4] = {0.f, 0.f, 0.f, 0.f};
+            const uint8_t* rowa = kcodes + (int64_t)ta * p.L.kc;
+            const uint8_t* rowb = kcodes + (int64_t)tb * p.L.kc;
+            const int swa = row_swizzle(KK, D, ta), swb = row_swizzle(KK, D, tb);
+#pragma unroll
+            for (int c = 0; c < T::KSTEPS / T::KCH; c++) {
+                const int lb = (T::KCW * c + 4 * T::KCH * j) * T::KBITS / 8;
+                Bytes<T::KNB> ka = lds_row<T::KNB>(rowa, lb, swa);
+                Bytes<T::KNB> kb = lds_row<T::KNB>(rowb, lb, swb);
+                uint32_t sca = 0, scb = 0;
+                if constexpr (KK == RK_E2M1_G16) {
+                    const int g = (T::KCW * c + 16 * j) / 16;
+                    sca = f16_splat(dec_e4m3x2_f16x2(kscl[ta * p.L.ks + g]));
+                    scb = f16_splat(dec_e4m3x2_f16x2(kscl[tb * p.L.ks + g]));
+                }
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int ks = 0; ks < T::KCH; ks++) {
+                    const int st = c * T::KCH + ks;
+                    uint32_t a[4];
+                    codes4_f16<KK, T::KNB>(ka, ks, a[0], a[2]);
+                    codes4_f16<KK, T::KNB>(kb, ks, a[1], a[3]);
+                    if constexpr (KK == RK_E2M1_G16) {
+                        a[0] = hmul2(a[0], sca); a[2] = hmul2(a[2], sca);
+                        a[1] = hmul2(a[1], scb); a[3] = hmul2(a[3], scb);
+                    }
+                    if constexpr (KK == RK_BF16RAW) {
+                        mma_bf16(acc, a, qh[st][0], qh[st][1]);
+                        mma_bf16(acc, a, ql[st][0], ql[st][1]);
+                    } else {
+                        mma_f16(acc, a, qh[st][0], qh[st][1]);
+                        mma_f16(acc, a, ql[st][0], ql[st][1]);
+                    }
+                }
+                if constexpr (KK == RK_INT8_G64 || KK == RK_E4M3_MX32) {
+                    float fa, fb;
+                    if constexpr (KK == RK_INT8_G64) {
+                        const uint16_t* s16 = reinterpret_cast<const uint16_t*>(kscl);
+                        fa = f16_bits_to_f32(s16[ta * (p.L.ks / 2) + c]);
+                        fb = f16_bits_to_f32(s16[tb * (p.L.ks / 2) + c]);
+                    } else {
+                        fa = ue8m0_to_f32(kscl[ta * p.L.ks + c]);
+                        fb = ue8m0_to_f32(kscl[tb * p.L.ks + c]);
+                    }
+                    sc[0] = fmaf(acc[0], fa, sc[0]);
+                    sc[1] = fmaf(acc[1], fa, sc[1]);
+                    sc[2] = fmaf(acc[2], fb, sc[2]);
+                    sc[3] = fmaf(acc[3], fb, sc[3]);
+                } else {
+                    sc[0] += acc[0]; sc[1] += acc[1]; sc[2] += acc[2]; sc[3] += acc[3];
+                }
+            }
+            if constexpr (KK == RK_E4M3_ROW256) {
+                const uint16_t* s16 = reinterpret_cast<const uint16_t*>(kscl);
+                const float fa = f16_bits_to_f32(s16[ta * (p.L.ks / 2)]);
+                const float fb = f16_bits_to_f32(s16[tb * (p.L.ks / 2)]);
+                sc[0] *= fa; sc[1] *= fa; sc[2] *= fb; sc[3] *= fb;
+            }
+            if (r >= valid) sc[0] = sc[1] = -INFINITY;
+            if (r + 8 >= valid) sc[2] = sc[3] = -INFINITY;
+
+            // ---------- online softmax (log2 domain), heads 2j and 2j+1
+            float x0 = fmaxf(sc[0], sc[2]), x1 = fmaxf(sc[1], sc[3]);
+#pragma unroll
+            for (int m = 4; m < 32; m <<= 1) {
+                x0 = fmaxf(x0, __shfl_xor_sync(0xffffffffu, x0, m));
+                x1 = fmaxf(x1, __shfl_xor_sync(0xffffffffu, x1, m));
+            }
+            const float n0 = fmaxf(m0, x0), n1 = fmaxf(m1, x1);
+            if (__any_sync(0xffffffffu, (n0 > m0) || (n1 > m1))) {
+                const float a0 = (m0 == -INFINITY) ? 0.f : exp2f(m0 - n0);
+                const float a1 = (m1 == -INFINITY) ? 0.f : exp2f(m1 - n1);
+#pragma unroll
+                for (int u = 0; u < T::DTILES; u++) {
+                    o[u][0] *= a0; o[u][1] *= a1; o[u][2] *= a0; o[u][3] *= a1;
+                }
+                l0 *= a0;
+                l1 *= a1;
+                m0 = n0;
+                m1 = n1;
+            }
+            const float r0 = (m0 == -INFINITY) ? 0.f : m0, r1 = (m1 == -INFINITY) ? 0.f : m1;
+            const float p0 = exp2f(sc[0] - r0), p1 = exp2f(sc[1] - r1);
+            const float p2 = exp2f(sc[2] - r0), p3 = exp2f(sc[3] - r1);
+            l0 += p0 + p2;
+            l1 += p1 + p3;
+
+            // ---------- O^T += V^T P^T
+            const uint8_t* vrowa = vcodes + (int64_t)ta * p.L.vc;
+            const uint8_t* vrowb = vcodes + (int64_t)tb * p.L.vc;
+            const int vswa = row_swizzle(KV, D, ta), vswb = row_swizzle(KV, D, tb);
+            uint32_t pb0 = 0, pb1 = 0;   // P'^T fragment (B operand)
+            if constexpr (KV == RK_E4M3_ROW256) {
+                const uint16_t* s16 = reinterpret_cast<const uint16_t*>(vscl);
+                const float fa = f16_bits_to_f32(s16[ta * (p.L.vs / 2)]);
+                const float fb = f16_bits_to_f32(s16[tb * (p.L.vs / 2)]);
+                pb0 = movtrans(pack_f16(p0 * fa, p1 * fa));
+                pb1 = movtrans(pack_f16(p2 * fb, p3 * fb));
+            } else if constexpr (KV != RK_INT8_G64 && KV != RK_E4M3_MX32) {
+                pb0 = movtrans(pack_f16(p0, p1));
+                pb1 = movtrans(pack_f16(p2, p3));
+            }
+#pragma unroll
+            for (int c = 0; c < T::DTILES / T::VCH; c++) {
+                if constexpr (KV == RK_INT8_G64 || KV == RK_E4M3_MX32) {
+                    float fa, fb;
+                    if constexpr (KV == RK_INT8_G64) {
+                        const uint16_t* s16 = reinterpret_cast<const uint16_t*>(vscl);
+                        fa = f16_bits_to_f32(s16[ta * (p.L.vs / 2) + c]);
+                        fb = f16_bits_to_f32(s16[tb * (p.L.vs / 2) + c]);
+                    } else {
+                        fa = ue8m0_to_f32(vscl[ta * p.L.vs + c]);
+                        fb = ue8m0_to_f32(vscl[tb * p.L.vs + c]);
+                    }
+                    pb0 = movtrans(pack_f16(p0 * fa, p1 * fa));
+                    pb1 = movtrans(pack_f16(p2 * fb, p3 * fb));
+                }
+                const int lb = (T::VCW * c + 4 * T::VCH * j) * T::VBITS / 8;
+                Bytes<T::VNB> va = lds_row<T::VNB>(vrowa, lb, vswa);
+                Bytes<T::VNB> vb = lds_row<T::VNB>(vrowb, lb, vswb);
+                uint32_t sva = 0, svb = 0;
+                if constexpr (KV == RK_E2M1_G16) {
+                    const int g = (T::VCW * c + 16 * j) / 16;
+                    sva = f16_splat(dec_e4m3x2_f16x2(vscl[ta * p.L.vs + g]));
+                    svb = f16_splat(dec_e4m3x2_f16x2(vscl[tb * p.L.vs + g]));
+                }
+#pragma unroll
+                for (int u = 0; u < T::VCH; u++) {
+                    uint32_t xa01, xa23, xb01, xb23;
+                    codes4_f16<KV, T::VNB>(va, u, xa01, xa23);
+                    codes4_f16<KV, T::VNB>(vb, u, xb01, xb23);
+                    if constexpr (KV == RK_E2M1_G16) {
+                        xa01 = hmul2(xa01, sva); xa23 = hmul2(xa23, sva);
+                        xb01 = hmul2(xb01, svb); xb23 = hmul2(xb23, svb);
+                    }
+                    uint32_t a[4] = {movtrans(xa01), movtrans(xa23), movtrans(xb01), movtrans(xb23)};
+                    mma_f16(o[c * T::VCH + u], a, pb0, pb1);
+                }
+            }
+        }
+
+        const bool seg_end = (i == n - 1) || (cc.page == cc.npages - 1);
+        __syncthreads();   // every warp is done with stage s (and with osm)
+        if (flags[0]) {
+            i_stop = i + 1;
+            break;
+        }
+        if (tid == 0 && issued < n) {
+            issue(s);
+            cursor_next(pc, pref, B, HH);
+            issued++;
+        }
+
+        if (seg_end) {
+            // ---- merge the four warps: max, rescaled sums, rescaled outputs
+#pragma unroll
+            for (int m = 4; m < 32; m <<= 1) {
+                l0 += __shfl_xor_sync(0xffffffffu, l0, m);
+                l1 += __shfl_xor_sync(0xffffffffu, l1, m);
+            }
+            if (r == 0) {
+                wml[warp * 16 + 2 * j] = m0;
+                wml[warp * 16 + 2 * j + 1] = m1;
+                wml[warp * 16 + 8 + 2 * j] = l0;
+                wml[warp * 16 + 8 + 2 * j + 1] = l1;
+            }
+            __syncthreads();
+            float M0 = -INFINITY, M1 = -INFINITY;
+#pragma unroll
+            for (int w = 0; w < 4; w++) {
+                M0 = fmaxf(M0, wml[w * 16 + 2 * j]);
+                M1 = fmaxf(M1, wml[w * 16 + 2 * j + 1]);
+            }
+            const float f0 = (m0 == -INFINITY) ? 0.f : exp2f(m0 - M0);
+            const float f1 = (m1 == -INFINITY) ? 0.f : exp2f(m1 - M1);
+            if (tid < 8) {
+                float M = -INFINITY, Ls = 0.f;
+                for (int w = 0; w < 4; w++) M = fmaxf(M, wml[w * 16 + tid]);
+                for (int w = 0; w < 4; w++) {
+                    float mw = wml[w * 16 + tid];
+                    if (mw != -INFINITY) Ls += exp2f(mw - M) * wml[w * 16 + 8 + tid];
+                }
+                fin[tid] = M;
+                fin[8 + tid] = Ls;
+            }
+            for (int w = 0; w < 4; w++) {
+                if (warp == w) {
+#pragma unroll
+                    for (int u = 0; u < T::DTILES; u++) {
+                        const int c = u / T::VCH, uu = u % T::VCH;
+                        const int base = T::VCW * c + 4 * uu;
+                        const int da = base + 4 * T::VCH * (r >> 1) + (r & 1);   // logical row r
+                        const int db = da + 2;                                    // logical row r + 8
+                        float* oa0 = osm + (2 * j) * D;
+                        float* oa1 = osm + (2 * j + 1) * D;
+                        if (w == 0) {
+                            oa0[da] = o[u][0] * f0; oa1[da] = o[u][1] * f1;
+                            oa0[db] = o[u][2] * f0; oa1[db] = o[u][3] * f1;
+                        } else {
+                            oa0[da] += o[u][0] * f0; oa1[da] += o[u][1] * f1;
+                            oa0[db] += o[u][2] * f0; oa1[db] += o[u][3] * f1;
+                        }
+                    }
+                }
+                __syncthreads();
+            }
+
+            // ---- full segment, or partial + arrival counter
+            const int64_t seg_w0 = (int64_t)pref[b] * HH + (int64_t)cc.hh * cc.npages;
+            const bool whole = (seg_w0 >= w0) && (seg_w0 + cc.npages <= w1);
+            bool emit = whole;
+            if (!whole) {
+                const int slot = seg_first ? 0 : 1;
+                float* part = p.partials + ((int64_t)blockIdx.x * 2 + slot) * (8 * (D + 2));
+                for (int x = tid; x < 16; x += kDecThreads) part[x] = fin[x];
+                for (int x = tid; x < 8 * D; x += kDecThreads) part[16 + x] = osm[x];
+                __threadfence();
+                __syncthreads();
+                const int i_first = owner_of(seg_w0, W, G);
+                const int i_last = owner_of(seg_w0 + cc.npages - 1, W, G);
+                int* ctr = p.counters + (int64_t)b * HH + cc.hh;
+                if (tid == 0) {
+                    int old = atomicAdd(ctr, 1);
+                    flags[1] = (old == i_last - i_first);
+                }
+                __syncthreads();
+                emit = flags[1] != 0;
+                if (emit) {
+                    __threadfence();
+                    // merge all partials of this segment (CTAs i_first .. i_last)
+                    if (tid < 8) {
+                        float M = -INFINITY;
+                        for (int k = i_first; k <= i_last; k++) {
+                            const int64_t sk = (int64_t)k * W / G;
+                            const float* pk = p.partials + ((int64_t)k * 2 + (sk >= seg_w0 ? 0 : 1)) * (8 * (D + 2));
+                            M = fmaxf(M, __ldcg(pk + tid));
+                        }
+                        float Ls = 0.f;
+                        for (int k = i_first; k <= i_last; k++) {
+                            const int64_t sk = (int64_t)k * W / G;
+                            const float* pk = p.partials + ((int64_t)k * 2 + (sk >= seg_w0 ? 0 : 1)) * (8 * (D + 2));
+                            const float mk = __ldcg(pk + tid);
+                            if (mk != -INFINITY) Ls += exp2f(mk - M) * __ldcg(pk + 8 + tid);
+                        }
+                        fin[tid] = M;
+                        fin[8 + tid] = Ls;
+                    }
+                    __syncthreads();
+                    for (int x = tid; x < 8 * D; x += kDecThreads) {
+                        const int g = x / D;
+                        const float M = fin[g];
+                        float acc = 0.f;
+                        for (int k = i_first; k <= i_last; k++) {
+                            const int64_t sk = (int64_t)k * W / G;
+                            const float* pk = p.partials + ((int64_t)k * 2 + (sk >= seg_w0 ? 0 : 1)) * (8 * (D + 2));
+                            const float mk = __ldcg(pk + g);
+                            if (mk != -INFINITY) acc += exp2f(mk - M) * __ldcg(pk + 16 + x);
+                        }
+                        osm[x] = acc;
+                    }
+                    if (tid == 0) *ctr = 0;
+                    __syncthreads();
+                }
+            }
+            if (emit) {
+                // ---- normalise, undo the V rotation, store
+#pragma unroll
+                for (int k = 0; k < 2; k++) {
+                    const int nh = warp + 4 * k;
+                    const int gq = hb * 8 + nh;
+                    if (gq < p.G) {
+                        const float Ls = fin[8 + nh];
+                        const float inv = (Ls > 0.f) ? p.o_mult / Ls : 0.f;
+                        float x[8];
+#pragma unroll
+                        for (int e = 0; e < T::EPL; e++) x[e] = osm[nh * D + lane * T::EPL + e] * inv;
+                        if constexpr (D == 256) {
+                            if (p.rot_v) fwht256_warp(x, lane);
+                        }
+                        const int64_t ob = ((int64_t)b * p.Hq + h * p.G + gq) * D + lane * T::EPL;
+                        if (p.out_fp32) {
+                            float* dst = reinterpret_cast<float*>(p.out) + ob;
+#pragma unroll
+                            for (int e = 0; e < T::EPL; e += 4)
+                                *reinterpret_cast<float4*>(dst + e) = make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]);
+                        } else {
+                            uint32_t w4[4];
+#pragma unroll
+                            for (int e = 0; e < T::EPL; e += 2) w4[e / 2] = pack_bf16(x[e], x[e + 1]);
+                            uint16_t* dst = reinterpret_cast<uint16_t*>(p.out) + ob;
+                            if constexpr (T::EPL == 8)
+                                *reinterpret_cast<uint4*>(dst) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                            else
+                                *reinterpret_cast<uint2*>(dst) = make_uint2(w4[0], w4[1]);
+                        }
+                    }
+                }
+            }
+            __syncthreads();   // osm and fin are free again
+        }
+        cursor_next(cc, pref, B, HH);
+    }
+
+    if (flags[0] && tid == 0) {
+        // a wait gave up: wait (bounded) for the copies still in flight before exiting
+        for (int k = i_stop; k < issued; k++)
+            (void)mbar_wait(smem_u32(&bars[k % NS]), (uint32_t)((k / NS) & 1));
+    }
+}
+
+// ------------------------------------------------------------ host side
+
+template <int KK, int KV, int D>
+static const void* kernel_ptr() {
+    return reinterpret_cast<const void*>(&decode_kernel<KK, KV, D>);
+}
+
+static const void* decode_kernel_for(int fmt, int D) {
+    const int kk = kind_of(fmt, 0), vk = kind_of(fmt, 1);
+#define KVQ_CASE(KK, KV)                                   \
+    if (kk == KK && vk == KV) {                            \
+        if (D == 256) return kernel_ptr<KK, KV, 256>();    \
+        if (D == 128) return kernel_ptr<KK, KV, 128>();    \
+    }
+    KVQ_CASE(RK_BF16RAW, RK_FP16)
+    KVQ_CASE(RK_E4M3_ROW256, RK_E4M3_ROW256)
+    KVQ_CASE(RK_INT8_G64, RK_INT8_G64)
+    KVQ_CASE(RK_E2M1_G16, RK_E2M1_G16)
+    KVQ_CASE(RK_E4M3_ROW256, RK_E2M1_G16)
+    KVQ_CASE(RK_E4M3_MX32, RK_E4M3_MX32)
+    KVQ_CASE(RK_E4M3_TENSOR, RK_E4M3_TENSOR)
+#undef KVQ_CASE
+    return nullptr;
+}
+
+bool decode_supported(int fmt, int D) {
+    if (fmt == F_FP8_ROW256 || fmt == F_K8V4) return D == 256;
+    return D == 128 || D == 256;
+}
+
+static size_t fixed_smem(int D, int B) {
+    return 8 * kMaxStages + 8 * (size_t)D * 4 + 4 * 16 * 4 + 16 * 4 + 16 + 4 * (size_t)(B + 1) + 128;
+}
+
+cudaError_t plan_decode(const Layout& L, int B, int HB, int max_seq_len, DecodePlan* plan) {
+    if (B > kMaxBatch) return cudaErrorInvalidValue;
+    int dev = 0, sms = 0, smem_sm = 0, smem_blk = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&smem_blk, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess) return e;
+    const size_t fixed = fixed_smem(L.D, B);
+    int ctas = 2;
+    int64_t stages = ((int64_t)smem_sm / 2 - 1024 - (int64_t)fixed) / L.slab;
+    if (stages < 3) {
+        ctas = 1;
+        stages = ((int64_t)smem_blk - (int64_t)fixed) / L.slab;
+    }
+    if (stages < 2) return cudaErrorInvalidValue;
+    if (stages > 6) stages = 6;
+    plan->stages = (int)stages;
+    plan->threads = kDecThreads;
+    plan->smem = (((size_t)stages * L.slab + 127) & ~(size_t)127) + fixed;
+    const int64_t pages = (max_seq_len + L.P - 1) / L.P;
+    int64_t work = (int64_t)B * pages * L.H * HB;
+    int64_t grid = (int64_t)sms * ctas;
+    if (work < grid) grid = work;
+    if (grid < 1) grid = 1;
+    plan->grid = (int)grid;
+    return cudaSuccess;
+}
+
+size_t decode_workspace_bytes(const Layout& L, int B, int HB, int grid) {
+    size_t partials = (size_t)grid * 2 * 8 * (L.D + 2) * sizeof(float);
+    size_t counters = (size_t)B * L.H * HB * sizeof(int);
+    return ((partials + 255) & ~(size_t)255) + ((counters + 255) & ~(size_t)255);
+}
+
+cudaError_t launch_decode(const DecodeParams& p, const DecodePlan& plan, cudaStream_t s) {
+    const void* k = decode_kernel_for(p.L.fmt, p.L.D);
+    if (!k) return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan.smem);
+    if (e != cudaSuccess) return e;
+    void* args[] = {const_cast<DecodeParams*>(&p)};
+    return cudaLaunchKernel(k, dim3(plan.grid), dim3(plan.threads), args, plan.smem, s);
+}
+
+}  // namespace kvq

@@ -1,0 +1,72 @@
+// kvq_internal.h -- kernel parameter blocks and launchers used by the C-ABI layer.
+#pragma once
+
+#include "kvq_common.cuh"
+
+namespace kvq {
+
+struct AppendParams {
+    Layout L;
+    uint8_t* slabs;              // first slab of the layer
+    const uint16_t* k;           // bf16 [n_tokens][H][D]
+    const uint16_t* v;
+    const int64_t* slots;
+    int n_tokens;
+    bool rot_k, rot_v;
+    float k_scale, v_scale;      // per-tensor scales (FP8_TENSOR)
+    uint32_t* status;
+};
+
+struct ReadParams {
+    Layout L;
+    const uint8_t* slabs;
+    const int64_t* slots;
+    int n;
+    uint8_t *k_codes, *k_scales, *v_codes, *v_scales;
+};
+
+struct DequantParams {
+    Layout L;
+    const uint8_t* slabs;
+    const int64_t* slots;
+    int n;
+    float k_scale, v_scale;
+    float *k_out, *v_out;
+};
+
+struct DecodeParams {
+    Layout L;
+    const uint8_t* slabs;        // first slab of the layer
+    const uint16_t* q;           // bf16 [B][Hq][D]
+    int Hq, G, HB;               // query heads, GQA group, 8-head blocks per kv-head
+    const int32_t* block_table;
+    int max_pages;
+    const int32_t* seq_lens;
+    int B;
+    void* out;
+    int out_fp32;
+    float q_mult;                // softmax_scale * log2(e) * K tensor scale
+    float o_mult;                // V tensor scale (1 otherwise)
+    bool rot_k, rot_v;
+    float* partials;             // [gridDim.x][2][8 * (D + 2)]
+    int* counters;               // [B][H][HB], zero between calls
+    uint32_t* status;
+    int stages;                  // pipeline depth (page slabs in shared memory)
+};
+
+cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
+cudaError_t launch_read_rows(const ReadParams& p, cudaStream_t s);
+cudaError_t launch_dequant(const DequantParams& p, cudaStream_t s);
+cudaError_t launch_encode(int code, const float* x, int64_t n, uint8_t* out, cudaStream_t s);
+
+// Decode: grid / smem plan for a layout (host side), then the launch.
+struct DecodePlan {
+    int grid, stages, threads;
+    size_t smem;
+};
+cudaError_t plan_decode(const Layout& L, int B, int HB, int max_seq_len, DecodePlan* plan);
+size_t decode_workspace_bytes(const Layout& L, int B, int HB, int grid);
+cudaError_t launch_decode(const DecodeParams& p, const DecodePlan& plan, cudaStream_t s);
+bool decode_supported(int fmt, int D);
+
+}  // namespace kvq
