@@ -483,14 +483,17 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const DecodePara
             l1 += p1 + p3;
 
             // ---------- O^T += V^T P^T
+            // rows past seq_len hold bytes never written: keep them out of the
+            // product entirely (their P is 0, but 0 x NaN would still be NaN)
+            const bool oka = r < valid, okb = r + 8 < valid, partial = valid < 16;
             const uint8_t* vrowa = vcodes + (int64_t)ta * p.L.vc;
             const uint8_t* vrowb = vcodes + (int64_t)tb * p.L.vc;
             const int vswa = row_swizzle(KV, D, ta), vswb = row_swizzle(KV, D, tb);
             uint32_t pb0 = 0, pb1 = 0;   // P'^T fragment (B operand)
             if constexpr (KV == RK_E4M3_ROW256) {
                 const uint16_t* s16 = reinterpret_cast<const uint16_t*>(vscl);
-                const float fa = f16_bits_to_f32(s16[ta * (p.L.vs / 2)]);
-                const float fb = f16_bits_to_f32(s16[tb * (p.L.vs / 2)]);
+                const float fa = oka ? f16_bits_to_f32(s16[ta * (p.L.vs / 2)]) : 0.f;
+                const float fb = okb ? f16_bits_to_f32(s16[tb * (p.L.vs / 2)]) : 0.f;
                 pb0 = movtrans(pack_f16(p0 * fa, p1 * fa));
                 pb1 = movtrans(pack_f16(p2 * fb, p3 * fb));
             } else if constexpr (KV != RK_INT8_G64 && KV != RK_E4M3_MX32) {
@@ -509,6 +512,8 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const DecodePara
                         fa = ue8m0_to_f32(vscl[ta * p.L.vs + c]);
                         fb = ue8m0_to_f32(vscl[tb * p.L.vs + c]);
                     }
+                    fa = oka ? fa : 0.f;
+                    fb = okb ? fb : 0.f;
                     pb0 = movtrans(pack_f16(p0 * fa, p1 * fa));
                     pb1 = movtrans(pack_f16(p2 * fb, p3 * fb));
                 }
@@ -529,6 +534,10 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const DecodePara
                     if constexpr (KV == RK_E2M1_G16) {
                         xa01 = hmul2(xa01, sva); xa23 = hmul2(xa23, sva);
                         xb01 = hmul2(xb01, svb); xb23 = hmul2(xb23, svb);
+                    }
+                    if (partial) {
+                        if (!oka) xa01 = xa23 = 0u;
+                        if (!okb) xb01 = xb23 = 0u;
                     }
                     uint32_t a[4] = {movtrans(xa01), movtrans(xa23), movtrans(xb01), movtrans(xb23)};
                     mma_f16(o[c * T::VCH + u], a, pb0, pb1);
