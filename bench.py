@@ -1,0 +1,435 @@
+"""Benchmark: quantized paged KV append + decode attention on B200.
+
+One step = append one new token per sequence (quantise + store) and run the
+decode attention over every sequence's cache (all steps of the hot path), with
+the prefix already in the cache and all inputs resident in HBM.  The headline
+workload is INT8-G64 (batch 8, lengths uniform in [1024, 8192], 8 kv-heads,
+32 query heads, head_dim 256, 64-token pages); the other formats' workloads are
+reported under "formats".
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--quick]
+
+N > 1: launched by torchrun, one rank per GPU; every rank runs its own replica
+(the path has no exchange step), timings are the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from quantized_paged_kv_03_b200 import inputs as I   # noqa: E402
+
+METRIC = "quantized-KV paged decode attention: HBM GB/s, % of peak, tokens/s per format"
+HEADLINE_CONFIG = 1
+L2_FLUSH_BYTES = 256 << 20
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# ---------------------------------------------------------------- accounting
+
+def decode_bytes(w: I.Workload, token_bytes: int, out_bytes_per_elem: int = 4) -> int:
+    """Algorithmic bytes of one decode: KV pages read + q + out + block table + seq_lens."""
+    kv = int(w.seq_lens.astype(np.int64).sum()) * w.H * token_bytes
+    pages = int(((w.seq_lens.astype(np.int64) + w.P - 1) // w.P).sum())
+    return kv + w.B * w.Hq * w.D * 2 + w.B * w.Hq * w.D * out_bytes_per_elem + pages * 4 + w.B * 4
+
+
+def append_bytes(n_tokens: int, w: I.Workload, token_bytes: int) -> int:
+    """Algorithmic bytes of one append: bf16 K and V read, codes + scales written, slots."""
+    return n_tokens * w.H * (2 * w.D * 2 + token_bytes) + 8 * n_tokens
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    def __init__(self, path):
+        self.path, self.proc = path, None
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "--query-gpu=index,clocks.sm,clocks.max.sm,power.draw,"
+                 "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+                 "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_power_cap", "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self, device_index=0):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        rows = []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9 or not f[1].isdigit():
+                continue
+            if int(f[0]) != device_index:
+                continue
+            rows.append(f)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [int(r[1]) for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": int(rows[0][2]), "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- GPU arm
+
+class Arm:
+    """One workload on the GPU: cache with the prefix appended, step inputs in HBM."""
+
+    def __init__(self, cfg: int, fmt: str, seed_offset: int = 0):
+        import torch
+        import quantized_paged_kv_03_b200 as K
+        self.torch, self.K = torch, K
+        spec = I.CONFIGS[cfg]
+        seed = I.SEED_BASE + cfg + 1000 * seed_offset
+        self.w = w = I.make_workload(cfg, fmt=fmt, seed=seed)
+        self.fmt = fmt
+        self.tb = K.token_bytes(fmt, w.D)
+        scales = None
+        if fmt == "fp8_tensor":
+            scales = [(I.tensor_amax(w.k) / 448.0 or 1.0, I.tensor_amax(w.v) / 448.0 or 1.0)]
+        self.cache = K.KVCache(fmt, w.D, w.H, w.P, w.num_pages, 1, 0, scales)
+        dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+        kp, vp, sp = w.prefix()
+        step = 1 << 20
+        for i in range(0, len(sp), step):     # bulk prefill, untimed
+            self.cache.append(0, dev(kp[i:i + step]).view(torch.bfloat16),
+                              dev(vp[i:i + step]).view(torch.bfloat16), dev(sp[i:i + step]))
+        del kp, vp
+        kn, vn, sn = w.new_tokens()
+        self.h_k, self.h_v, self.h_s = kn, vn, sn
+        self.k_new = dev(kn).view(torch.bfloat16)
+        self.v_new = dev(vn).view(torch.bfloat16)
+        self.slots = dev(sn)
+        self.q = dev(w.q).view(torch.bfloat16)
+        self.bt = dev(w.block_table)
+        self.sl = dev(w.seq_lens)
+        self.out = torch.empty((w.B, w.Hq, w.D), dtype=torch.float32, device="cuda")
+        self.ws = self.cache.workspace(w.B, w.Hq, w.max_seq_len)
+        self.dec_bytes = decode_bytes(w, self.tb)
+        self.app_bytes = append_bytes(w.B, w, self.tb)
+        self.w.k = self.w.v = None     # host copies no longer needed
+        torch.cuda.synchronize()
+
+    def step(self):
+        self.cache.append(0, self.k_new, self.v_new, self.slots)
+        self.cache.decode_attention(0, self.q, self.bt, self.sl, self.w.max_seq_len, out=self.out,
+                                    workspace=self.ws)
+
+    def run(self, steps: int, warmup: int, flush):
+        """Device-timed steps: per step (append, decode) event pairs, L2 flushed
+        before each step outside the events."""
+        torch = self.torch
+        for _ in range(warmup):
+            flush()
+            self.step()
+        torch.cuda.synchronize()
+        s = torch.cuda.current_stream()
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+        for i in range(steps):
+            flush()
+            ev[i][0].record(s)
+            self.cache.append(0, self.k_new, self.v_new, self.slots)
+            ev[i][1].record(s)
+            self.cache.decode_attention(0, self.q, self.bt, self.sl, self.w.max_seq_len, out=self.out,
+                                        workspace=self.ws)
+            ev[i][2].record(s)
+        torch.cuda.synchronize()
+        app = np.array([e[0].elapsed_time(e[1]) for e in ev])
+        dec = np.array([e[1].elapsed_time(e[2]) for e in ev])
+        return app, dec
+
+    def run_e2e(self, steps: int, warmup: int, flush):
+        """Same step through the public API from pinned host buffers: H2D of the
+        step's inputs, append, decode, D2H of the output, all inside the events."""
+        torch = self.torch
+        pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()
+        hk, hv, hs = pin(self.h_k).view(torch.bfloat16), pin(self.h_v).view(torch.bfloat16), pin(self.h_s)
+        hq = pin(self.w.q).view(torch.bfloat16)
+        hbt, hsl = pin(self.w.block_table), pin(self.w.seq_lens)
+        hout = torch.empty(self.out.shape, dtype=torch.float32).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in (hk, hv, hs, hq, hbt, hsl))
+        d2h = hout.numel() * 4
+        s = torch.cuda.current_stream()
+
+        def one():
+            self.k_new.copy_(hk, non_blocking=True)
+            self.v_new.copy_(hv, non_blocking=True)
+            self.slots.copy_(hs, non_blocking=True)
+            self.q.copy_(hq, non_blocking=True)
+            self.bt.copy_(hbt, non_blocking=True)
+            self.sl.copy_(hsl, non_blocking=True)
+            self.step()
+            hout.copy_(self.out, non_blocking=True)
+
+        for _ in range(warmup):
+            flush()
+            one()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(steps):
+            flush()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(s)
+            one()
+            b.record(s)
+            b.synchronize()
+            ts.append(a.elapsed_time(b))
+        return np.array(ts), h2d, d2h
+
+
+# ---------------------------------------------------------------- oracle arm
+
+def oracle_sample(cfg: int, fmt: str, budget_s: float = 12.0, threads: int | None = None):
+    """Time the CPU oracle (as it stands) on a bounded sample of one step of the
+    workload: the step's appends plus the decode of as many (sequence, kv-head)
+    jobs as fit in about `budget_s`; returns GB/s of the same algorithmic bytes."""
+    from concurrent.futures import ThreadPoolExecutor
+    import oracle as O
+    threads = threads or min(32, os.cpu_count() or 1)
+    w = I.make_workload(cfg, fmt=fmt)
+    f = {v: k for k, v in O.FORMAT_NAMES.items()}[fmt]
+    tb = O.token_bytes(f, w.D)
+    G = w.Hq // w.H
+    scale = 1.0 / np.sqrt(w.D)
+    # per-job inputs prepared outside the timing: bf16 rows of each (b, h)
+    jobs = [(b, h) for b in range(w.B) for h in range(w.H)]
+    rng = np.random.default_rng(0)
+    rng.shuffle(jobs)
+
+    def job(bh):
+        b, h = bh
+        rows = slice(int(w.starts[b]), int(w.starts[b + 1]))
+        kc, ks = O.quantize_rows(f, False, w.k[rows, h])
+        vc, vs = O.quantize_rows(f, True, w.v[rows, h])
+        kd = O.dequant_rows(f, False, kc, ks, w.D)
+        vd = O.dequant_rows(f, True, vc, vs, w.D)
+        q = O.bf16_bits_to_f64(w.q[b, h * G:(h + 1) * G])
+        O.attend(q, kd, vd, O.is_rotated(f, False), O.is_rotated(f, True), scale)
+        return int(w.seq_lens[b])
+
+    t0 = time.perf_counter()
+    done_tokens = 0
+    done = 0
+    with ThreadPoolExecutor(threads) as ex:
+        # cycle through the step's jobs until the time budget is used (at least one pass)
+        while done < len(jobs) or time.perf_counter() - t0 < budget_s:
+            batch = [jobs[(done + i) % len(jobs)] for i in range(threads)]
+            done_tokens += sum(ex.map(job, batch))
+            done += len(batch)
+    dt = time.perf_counter() - t0
+    # bytes of the decode work done (the quantisation of the rows stands in for
+    # the step's append of those rows and is not counted)
+    nbytes = done_tokens * tb + done * G * w.D * (2 + 4)
+    return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": f"{done} (sequence, kv-head) decode jobs cycling over the {len(jobs)} of one step of "
+                      f"{I.CONFIGS[cfg].name} ({done_tokens} cached tokens quantised, dequantised and "
+                      f"attended in fp64) in {dt:.1f} s on {threads} threads"}
+
+
+# ---------------------------------------------------------------- main
+
+def dist_setup(n):
+    if n <= 1:
+        return 0, 1, None
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", str(n)))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    torch.cuda.set_device(local)
+    dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    return rank, world, dist
+
+
+def max_over_ranks(x: float, dist) -> float:
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, dist) -> float:
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def reference_arm(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    fmt = I.CONFIGS[HEADLINE_CONFIG].formats[0]
+    budget = max(2.0, 10.0 * args.steps / max(1, args.steps + args.warmup))
+    vals = []
+    last = None
+    for _ in range(args.warmup):
+        oracle_sample(HEADLINE_CONFIG, fmt, budget_s=1.0)
+    for _ in range(args.steps):
+        last = oracle_sample(HEADLINE_CONFIG, fmt, budget_s=budget)
+        vals.append(last["value"])
+    v = float(np.mean(vals))
+    spec = I.CONFIGS[HEADLINE_CONFIG]
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": spec.name, "format": fmt},
+            "cpu_baseline": {"value": v, "unit": "GB/s", "cores": last["cores"], "kind": "oracle",
+                             "sample": last["sample"]},
+            "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--quick", action="store_true", help="headline workload only")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the oracle baseline")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return reference_arm(args)
+
+    import torch
+    from quantized_paged_kv_03_b200 import build
+    rank, world, dist = dist_setup(args.gpus)
+    if rank == 0:
+        build.build()
+    if dist is not None:
+        dist.barrier()
+    peak, peak_kind = load_peaks()
+    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    flush = lambda: flush_buf.fill_(1)
+
+    spec = I.CONFIGS[HEADLINE_CONFIG]
+    fmt = spec.formats[0]
+    arm = Arm(HEADLINE_CONFIG, fmt, seed_offset=rank)
+    clocks_path = os.path.join(ROOT, "gpurun_out", f"bench_clocks_r{rank}.csv")
+    os.makedirs(os.path.dirname(clocks_path), exist_ok=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(clocks_path) as clk:
+        t_wall = time.perf_counter()
+        app, dec = arm.run(args.steps, args.warmup, flush)
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        t_wall = time.perf_counter() - t_wall
+    step_ms = float((app + dec).mean())
+    dec_ms = float(dec.mean())
+    step_ms_max = max_over_ranks(step_ms, dist)
+    dec_ms_max = max_over_ranks(dec_ms, dist)
+    step_bytes = arm.dec_bytes + arm.app_bytes
+    total_bytes = sum_over_ranks(step_bytes, dist)
+    value = total_bytes / (step_ms_max * 1e-3) / 1e9
+    tokens = sum_over_ranks(arm.w.B, dist) / (step_ms_max * 1e-3)
+
+    e2e_ts, h2d, d2h = arm.run_e2e(max(5, args.steps // 2), args.warmup, flush)
+    e2e_ms = max_over_ranks(float(e2e_ts.mean()), dist)
+    dec_gbs = arm.dec_bytes / (dec_ms_max * 1e-3) / 1e9
+
+    formats = {}
+    if not args.quick:
+        for cfg in (0, 2, 3, 4):
+            for f in I.CONFIGS[cfg].formats:
+                a = Arm(cfg, f, seed_offset=rank)
+                ap_, de_ = a.run(args.steps, args.warmup, flush)
+                dm = max_over_ranks(float(de_.mean()), dist)
+                am = max_over_ranks(float(ap_.mean()), dist)
+                formats[f"{I.CONFIGS[cfg].name}/{f}"] = {
+                    "decode_ms": round(dm, 5), "decode_GBps": round(a.dec_bytes / (dm * 1e-3) / 1e9, 1),
+                    "decode_pct_of_peak": round(100 * a.dec_bytes / (dm * 1e-3) / 1e9 / peak, 1),
+                    "decode_tokens_per_s": round(a.w.B / (dm * 1e-3), 1),
+                    "append_ms": round(am, 5), "append_GBps": round(a.app_bytes / (am * 1e-3) / 1e9, 1),
+                    "step_tokens_per_s": round(a.w.B / ((dm + am) * 1e-3), 1),
+                    "decode_bytes": a.dec_bytes, "bytes_per_token_head": a.tb}
+                del a
+                torch.cuda.empty_cache()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = oracle_sample(HEADLINE_CONFIG, fmt, budget_s=12.0)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms_max, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f16-mma/f32-acc (int8 codes)", "data": "synthetic",
+            "config": {"workload": spec.name, "format": fmt, "batch": arm.w.B,
+                       "n_kv_heads": arm.w.H, "n_q_heads": arm.w.Hq, "head_dim": arm.w.D,
+                       "page_size": arm.w.P, "kv_tokens": int(arm.w.seq_lens.sum()),
+                       "step": "append 1 token/sequence + decode attention",
+                       "l2": "flushed (256 MiB write) before every step, outside the timed events",
+                       "parallelism": f"replicas x{world}"},
+            "tokens_per_s": round(tokens, 1),
+            "pct_of_peak": round(100 * value / peak, 2),
+            "decode_GBps": round(dec_gbs, 1),
+            "roofline": {"bound": "hbm", "achieved": round(dec_gbs, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(dec_gbs / peak, 4), "traffic": None,
+                         "kernel": "decode_kernel (split-K paged GQA decode, one launch per step)",
+                         "peak_source": f"{peak_kind} hbm_gbs"},
+            "e2e": {"value": round(total_bytes / (e2e_ms * 1e-3) / 1e9 if world > 1 else
+                                   step_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                    "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": int(h2d),
+                    "d2h_bytes_per_step": int(d2h)},
+            "gpu_launches": 2 * args.steps,
+            "clocks": clk.summary(int(os.environ.get("LOCAL_RANK", "0"))),
+            "wall_s_timed_region": round(t_wall, 3),
+            "formats": formats,
+        }
+        if cpu is not None:
+            line["cpu_baseline"] = cpu
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
