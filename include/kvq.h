@@ -149,6 +149,31 @@ int kvq_decode_attention(kvq_cache* cache, int32_t layer, const void* q, int32_t
                          void* out, int32_t out_fp32, float softmax_scale,
                          void* workspace, size_t workspace_bytes, void* stream);
 
+/* Size of the fixed device scratch array used by kvq_decode_attention_noalloc. */
+#define KVQ_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+/* kvq_decode_attention without a caller-provided workspace.  This entry point
+ * has no counterpart on the pages: it exists for callers that cannot allocate
+ * device memory -- a plugin given only its input and output buffers by a host
+ * engine, a process under a fixed device-memory budget that forbids new
+ * allocations after start-up, or a latency-critical loop where cudaMalloc and
+ * cudaFree (which can synchronise the device) are not allowed.
+ *   Same arguments and results as kvq_decode_attention, minus the workspace.
+ *   Scratch: a file-scope device array of KVQ_NOALLOC_SCRATCH_BYTES (8 MiB) in
+ *   the library image; every GPU that loads the library holds it until the
+ *   process exits.  Sizes whose workspace (kvq_decode_workspace_bytes) exceeds
+ *   it are rejected with KVQ_ERR_WORKSPACE before any launch.
+ *   The first call on a device looks up the array's device address (once per
+ *   device, with that device current); make that first call before any stream
+ *   capture.  Each call clears the part of the array that must start at zero
+ *   (a memset on `stream`) and calls no allocating routine.
+ *   All calls share the one array: calls that overlap on the GPU (different
+ *   streams, or several host threads) race and corrupt each other's results. */
+int kvq_decode_attention_noalloc(kvq_cache* cache, int32_t layer, const void* q, int32_t n_q_heads,
+                                 const int32_t* block_table, int32_t max_pages_per_seq,
+                                 const int32_t* seq_lens, int32_t batch, int32_t max_seq_len,
+                                 void* out, int32_t out_fp32, float softmax_scale, void* stream);
+
 /* Test surface: stored values of the rows at `slots`, as fp32 code x scale in
  * the stored (rotated) domain.  k_out, v_out: fp32 [n][n_kv_heads][head_dim]. */
 int kvq_dequant(kvq_cache* cache, int32_t layer, const int64_t* slots, int32_t n,

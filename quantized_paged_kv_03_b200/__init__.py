@@ -23,6 +23,7 @@ FORMAT_NAMES = {v: k for k, v in FORMATS.items()}
 FLAG_NO_ROTATE = 1
 CODES = {"e4m3": 0, "e2m1": 1, "int8": 2, "fp16": 3, "ue4m3": 4}
 STATUS_BAD_SLOT, STATUS_BAD_PAGE, STATUS_WAIT_TIMEOUT = 1, 2, 4
+NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
 class KVQError(RuntimeError):
@@ -61,6 +62,8 @@ def lib() -> ctypes.CDLL:
         "kvq_decode_workspace_bytes": (sz, [P, i32, i32, i32]),
         "kvq_decode_attention": (ctypes.c_int, [P, i32, P, i32, P, i32, P, i32, i32, P, i32, f32,
                                                 P, sz, P]),
+        "kvq_decode_attention_noalloc": (ctypes.c_int, [P, i32, P, i32, P, i32, P, i32, i32, P, i32,
+                                                        f32, P]),
         "kvq_dequant": (ctypes.c_int, [P, i32, P, i32, P, P, P]),
         "kvq_read_rows": (ctypes.c_int, [P, i32, P, i32, P, P, P, P, P]),
         "kvq_encode": (ctypes.c_int, [i32, P, i64, P, P]),
@@ -79,7 +82,7 @@ def lib() -> ctypes.CDLL:
 def exported_symbols():
     return ["kvq_token_bytes", "kvq_row_bytes", "kvq_cache_bytes", "kvq_cache_create",
             "kvq_cache_destroy", "kvq_append", "kvq_decode_workspace_bytes",
-            "kvq_decode_attention", "kvq_dequant", "kvq_read_rows", "kvq_encode",
+            "kvq_decode_attention", "kvq_decode_attention_noalloc", "kvq_dequant", "kvq_read_rows", "kvq_encode",
             "kvq_read_device_status", "kvq_status_string", "kvq_version"]
 
 
@@ -237,6 +240,27 @@ class KVCache:
                                           _ptr(out), int(out_fp32), float(softmax_scale),
                                           _ptr(ws), ws.numel(), _stream(stream)),
                "decode_attention")
+        return out
+
+    def decode_attention_noalloc(self, layer: int, q, block_table, seq_lens, max_seq_len: int, out,
+                                 out_fp32: bool = True, softmax_scale: float = 0.0, stream=None):
+        """decode_attention for callers that cannot allocate device memory: the
+        scratch lives in a fixed 8 MiB array inside the library, so no workspace
+        is passed and nothing is allocated (the caller still provides `out`).
+        Calls that overlap on the GPU share that array and must not run
+        concurrently; the first call on a device should come before any stream
+        capture."""
+        import torch
+        _dev_tensor(q, torch.bfloat16, "q")
+        _dev_tensor(block_table, torch.int32, "block_table")
+        _dev_tensor(seq_lens, torch.int32, "seq_lens")
+        _dev_tensor(out, torch.float32 if out_fp32 else torch.bfloat16, "out")
+        B, Hq, D = q.shape
+        _check(lib().kvq_decode_attention_noalloc(self._h, layer, _ptr(q), Hq, _ptr(block_table),
+                                                  block_table.shape[1], _ptr(seq_lens), B, max_seq_len,
+                                                  _ptr(out), int(out_fp32), float(softmax_scale),
+                                                  _stream(stream)),
+               "decode_attention_noalloc")
         return out
 
     def dequant(self, layer: int, slots, stream=None):

@@ -18,6 +18,8 @@ struct kvq_cache {
     float* tensor_scales;   // host [num_layers][2]
 };
 
+const Layout* kvq_cache_layout(const kvq_cache* cache) { return cache ? &cache->L : nullptr; }
+
 static int desc_layout(const kvq_cache_desc* d, Layout* out) {
     if (!d) return KVQ_ERR_ARG;
     if (d->format < 0 || d->format >= F_COUNT) return KVQ_ERR_FORMAT;

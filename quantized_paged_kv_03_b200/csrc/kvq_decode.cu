@@ -783,6 +783,13 @@ size_t decode_workspace_bytes(const Layout& L, int B, int HB, int grid) {
     return ((partials + 255) & ~(size_t)255) + ((counters + 255) & ~(size_t)255);
 }
 
+void decode_workspace_zero_region(const Layout& L, int B, int HB, int grid, size_t* offset, size_t* bytes) {
+    size_t partials = (size_t)grid * 2 * 8 * (L.D + 2) * sizeof(float);
+    size_t counters = (size_t)B * L.H * HB * sizeof(int);
+    *offset = (partials + 255) & ~(size_t)255;
+    *bytes = (counters + 255) & ~(size_t)255;
+}
+
 cudaError_t launch_decode(const DecodeParams& p, const DecodePlan& plan, cudaStream_t s) {
     const void* k = decode_kernel_for(p.L.fmt, p.L.D);
     if (!k) return cudaErrorInvalidValue;

@@ -66,7 +66,13 @@ struct DecodePlan {
 };
 cudaError_t plan_decode(const Layout& L, int B, int HB, int max_seq_len, DecodePlan* plan);
 size_t decode_workspace_bytes(const Layout& L, int B, int HB, int grid);
+// Byte range of a decode workspace that must hold zeros when a call starts.
+void decode_workspace_zero_region(const Layout& L, int B, int HB, int grid, size_t* offset, size_t* bytes);
 cudaError_t launch_decode(const DecodeParams& p, const DecodePlan& plan, cudaStream_t s);
 bool decode_supported(int fmt, int D);
 
 }  // namespace kvq
+
+struct kvq_cache;
+// Page layout of a cache handle (defined with the handle in kvq_api.cu).
+const kvq::Layout* kvq_cache_layout(const kvq_cache* cache);
