@@ -189,9 +189,10 @@ int kvq_decode_attention(kvq_cache* cache, int32_t layer, const void* q, int32_t
     p.o_mult = cache->tensor_scales[2 * layer + 1];
     p.rot_k = rot_of(cache, 0);
     p.rot_v = rot_of(cache, 1);
-    const size_t part_bytes = ((size_t)plan.grid * 2 * 8 * (cache->L.D + 2) * sizeof(float) + 255) & ~(size_t)255;
+    size_t zoff = 0, zbytes = 0;
+    decode_workspace_zero_region(cache->L, batch, HB, plan.grid, &zoff, &zbytes);
     p.partials = (float*)workspace;
-    p.counters = (int*)((uint8_t*)workspace + part_bytes);
+    p.barrier = (unsigned*)((uint8_t*)workspace + zoff);
     p.status = (uint32_t*)cache->pool;
     p.stages = plan.stages;
     return cuda_status(launch_decode(p, plan, (cudaStream_t)stream));

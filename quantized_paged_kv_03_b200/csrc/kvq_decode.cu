@@ -37,7 +37,6 @@ namespace kvq {
 constexpr int kDecThreads = 128;
 constexpr int kMaxStages = 8;
 constexpr int kMaxBatch = 4096;
-constexpr float kLog2e = 1.4426950408889634f;
 
 // ------------------------------------------------------------ PTX helpers
 
@@ -196,6 +195,132 @@ __device__ __forceinline__ void cursor_locate(Cursor& c, int64_t w, const int* p
 // CTA owning page-head w when W page-heads are cut into G equal ranges.
 __device__ __forceinline__ int owner_of(int64_t w, int64_t W, int G) {
     return (int)(((w + 1) * G + W - 1) / W) - 1;
+}
+
+// Store EPL consecutive output values (fp32 or bf16) at element offset `ob`.
+template <int EPL>
+__device__ __forceinline__ void store_out(const DecodeParams& p, int64_t ob, const float* x) {
+    if (p.out_fp32) {
+        float* dst = reinterpret_cast<float*>(p.out) + ob;
+#pragma unroll
+        for (int e = 0; e < EPL; e += 4)
+            *reinterpret_cast<float4*>(dst + e) = make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]);
+    } else {
+        uint16_t* dst = reinterpret_cast<uint16_t*>(p.out) + ob;
+#pragma unroll
+        for (int e = 0; e < EPL; e += 4)
+            *reinterpret_cast<uint2*>(dst + e) = make_uint2(pack_bf16(x[e], x[e + 1]), pack_bf16(x[e + 2], x[e + 3]));
+    }
+}
+
+// Grid-wide barrier of the G co-resident CTAs (cooperative launch).  Arrival
+// counter + generation word in the workspace; the last arriver resets the
+// counter, so it is zero again after every launch.  The wait is bounded: on
+// timeout the CTA records it and returns false.
+__device__ __forceinline__ bool grid_barrier(unsigned* bar, unsigned G, int* flag_smem) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        volatile unsigned* vgen = bar + 1;
+        const unsigned gen = *vgen;
+        __threadfence();
+        const unsigned old = atomicAdd(bar, 1u);
+        int ok = 1;
+        if (old == G - 1) {
+            atomicExch(bar, 0u);
+            __threadfence();
+            atomicAdd(bar + 1, 1u);
+        } else {
+            long it = 0;
+            while (*vgen == gen) {
+                __nanosleep(64);
+                if (++it > (1l << 26)) {
+                    ok = 0;
+                    break;
+                }
+            }
+        }
+        __threadfence();
+        *flag_smem = ok;
+    }
+    __syncthreads();
+    return *flag_smem != 0;
+}
+
+// Merge share `j` of the partials of one cut segment (CTAs i_first..i_last
+// each left (max, sum, unnormalised output) for up to 8 query heads): this CTA
+// produces float4 outputs [o0, o1) of the segment's gv x D/4.
+template <int D>
+__device__ __forceinline__ void merge_segment(const DecodeParams& p, int b, int h, int hb, int64_t seg_w0,
+                                              int i_first, int i_last, int64_t W, int G, float* fin) {
+    const int tid = threadIdx.x;
+    const int P = i_last - i_first + 1;
+    const int j = (int)blockIdx.x - i_first;
+    const int gv = min(8, p.G - hb * 8);
+    const int NU = gv * (D / 4);
+    const int o0 = (int)((int64_t)j * NU / P), o1 = (int)((int64_t)(j + 1) * NU / P);
+    auto part_of = [&](int k) -> const float* {
+        const int i = i_first + k;
+        const int64_t start = (int64_t)i * W / G;
+        return p.partials + ((int64_t)i * 2 + (start >= seg_w0 ? 0 : 1)) * (16 + 8 * D);
+    };
+    // segment max and sum per head: 16 lanes per head
+    {
+        const int g = tid >> 4, pl = tid & 15;
+        float M = -INFINITY;
+        for (int k = pl; k < P; k += 16) M = fmaxf(M, __ldcg(part_of(k) + g));
+#pragma unroll
+        for (int m = 1; m < 16; m <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, m));
+        float L = 0.f;
+        for (int k = pl; k < P; k += 16) {
+            const float* pk = part_of(k);
+            const float mk = __ldcg(pk + g);
+            if (mk != -INFINITY) L += exp2f(mk - M) * __ldcg(pk + 8 + g);
+        }
+#pragma unroll
+        for (int m = 1; m < 16; m <<= 1) L += __shfl_xor_sync(0xffffffffu, L, m);
+        __syncthreads();
+        if (pl == 0) {
+            fin[g] = M;
+            fin[8 + g] = L;
+        }
+        __syncthreads();
+    }
+    const int no = o1 - o0;
+    if (no <= 0) return;
+    int tpo = 1;
+    while (tpo < 16 && tpo * 2 * no <= kDecThreads) tpo *= 2;
+    const int per_pass = kDecThreads / tpo;
+    for (int ob = o0; ob < o1; ob += per_pass) {
+        const int o = ob + tid / tpo, pl = tid % tpo;
+        const bool valid = o < o1;
+        const int g = valid ? o / (D / 4) : 0, d4 = valid ? o % (D / 4) : 0;
+        const float M = fin[g];
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (valid) {
+            for (int k = pl; k < P; k += tpo) {
+                const float* pk = part_of(k);
+                const float mk = __ldcg(pk + g);
+                const float4 v = __ldcg(reinterpret_cast<const float4*>(pk + 16 + g * D) + d4);
+                const float wk = (mk == -INFINITY) ? 0.f : exp2f(mk - M);
+                acc.x = fmaf(wk, v.x, acc.x); acc.y = fmaf(wk, v.y, acc.y);
+                acc.z = fmaf(wk, v.z, acc.z); acc.w = fmaf(wk, v.w, acc.w);
+            }
+        }
+        for (int m = 1; m < tpo; m <<= 1) {
+            acc.x += __shfl_xor_sync(0xffffffffu, acc.x, m);
+            acc.y += __shfl_xor_sync(0xffffffffu, acc.y, m);
+            acc.z += __shfl_xor_sync(0xffffffffu, acc.z, m);
+            acc.w += __shfl_xor_sync(0xffffffffu, acc.w, m);
+        }
+        if (valid && pl == 0) {
+            const float Ls = fin[8 + g];
+            const float inv = (Ls > 0.f) ? p.o_mult / Ls : 0.f;
+            const float x[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
+            const int64_t oo = ((int64_t)b * p.Hq + h * p.G + hb * 8 + g) * D + 4 * d4;
+            store_out<4>(p, oo, x);
+        }
+    }
+    __syncthreads();
 }
 
 template <int KK, int KV, int D>
@@ -611,94 +736,35 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const DecodePara
                 __syncthreads();
             }
 
-            // ---- full segment, or partial + arrival counter
+            // ---- a whole segment is normalised and stored here; a segment cut by
+            // a range boundary leaves its unnormalised output as this CTA's partial
+            // (rotated back already: the Hadamard is linear, so merging commutes
+            // with it) for the merge after the grid barrier.
             const int64_t seg_w0 = (int64_t)pref[b] * HH + (int64_t)cc.hh * cc.npages;
             const bool whole = (seg_w0 >= w0) && (seg_w0 + cc.npages <= w1);
-            bool emit = whole;
-            if (!whole) {
-                const int slot = seg_first ? 0 : 1;
-                float* part = p.partials + ((int64_t)blockIdx.x * 2 + slot) * (8 * (D + 2));
-                for (int x = tid; x < 16; x += kDecThreads) part[x] = fin[x];
-                for (int x = tid; x < 8 * D; x += kDecThreads) part[16 + x] = osm[x];
-                __threadfence();
-                __syncthreads();
-                const int i_first = owner_of(seg_w0, W, G);
-                const int i_last = owner_of(seg_w0 + cc.npages - 1, W, G);
-                int* ctr = p.counters + (int64_t)b * HH + cc.hh;
-                if (tid == 0) {
-                    int old = atomicAdd(ctr, 1);
-                    flags[1] = (old == i_last - i_first);
-                }
-                __syncthreads();
-                emit = flags[1] != 0;
-                if (emit) {
-                    __threadfence();
-                    // merge all partials of this segment (CTAs i_first .. i_last)
-                    if (tid < 8) {
-                        float M = -INFINITY;
-                        for (int k = i_first; k <= i_last; k++) {
-                            const int64_t sk = (int64_t)k * W / G;
-                            const float* pk = p.partials + ((int64_t)k * 2 + (sk >= seg_w0 ? 0 : 1)) * (8 * (D + 2));
-                            M = fmaxf(M, __ldcg(pk + tid));
-                        }
-                        float Ls = 0.f;
-                        for (int k = i_first; k <= i_last; k++) {
-                            const int64_t sk = (int64_t)k * W / G;
-                            const float* pk = p.partials + ((int64_t)k * 2 + (sk >= seg_w0 ? 0 : 1)) * (8 * (D + 2));
-                            const float mk = __ldcg(pk + tid);
-                            if (mk != -INFINITY) Ls += exp2f(mk - M) * __ldcg(pk + 8 + tid);
-                        }
-                        fin[tid] = M;
-                        fin[8 + tid] = Ls;
-                    }
-                    __syncthreads();
-                    for (int x = tid; x < 8 * D; x += kDecThreads) {
-                        const int g = x / D;
-                        const float M = fin[g];
-                        float acc = 0.f;
-                        for (int k = i_first; k <= i_last; k++) {
-                            const int64_t sk = (int64_t)k * W / G;
-                            const float* pk = p.partials + ((int64_t)k * 2 + (sk >= seg_w0 ? 0 : 1)) * (8 * (D + 2));
-                            const float mk = __ldcg(pk + g);
-                            if (mk != -INFINITY) acc += exp2f(mk - M) * __ldcg(pk + 16 + x);
-                        }
-                        osm[x] = acc;
-                    }
-                    if (tid == 0) *ctr = 0;
-                    __syncthreads();
-                }
-            }
-            if (emit) {
-                // ---- normalise, undo the V rotation, store
+            float* part = p.partials + ((int64_t)blockIdx.x * 2 + (seg_first ? 0 : 1)) * (16 + 8 * D);
+            if (!whole && tid < 16) part[tid] = fin[tid];
 #pragma unroll
-                for (int k = 0; k < 2; k++) {
-                    const int nh = warp + 4 * k;
-                    const int gq = hb * 8 + nh;
-                    if (gq < p.G) {
-                        const float Ls = fin[8 + nh];
-                        const float inv = (Ls > 0.f) ? p.o_mult / Ls : 0.f;
-                        float x[8];
+            for (int k = 0; k < 2; k++) {
+                const int nh = warp + 4 * k;
+                const int gq = hb * 8 + nh;
+                if (gq < p.G) {
+                    const float Ls = fin[8 + nh];
+                    const float inv = whole ? ((Ls > 0.f) ? p.o_mult / Ls : 0.f) : 1.f;
+                    float x[8];
 #pragma unroll
-                        for (int e = 0; e < T::EPL; e++) x[e] = osm[nh * D + lane * T::EPL + e] * inv;
-                        if constexpr (D == 256) {
-                            if (p.rot_v) fwht256_warp(x, lane);
-                        }
+                    for (int e = 0; e < T::EPL; e++) x[e] = osm[nh * D + lane * T::EPL + e] * inv;
+                    if constexpr (D == 256) {
+                        if (p.rot_v) fwht256_warp(x, lane);
+                    }
+                    if (!whole) {
+                        float* dst = part + 16 + nh * D + lane * T::EPL;
+#pragma unroll
+                        for (int e = 0; e < T::EPL; e += 4)
+                            *reinterpret_cast<float4*>(dst + e) = make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]);
+                    } else {
                         const int64_t ob = ((int64_t)b * p.Hq + h * p.G + gq) * D + lane * T::EPL;
-                        if (p.out_fp32) {
-                            float* dst = reinterpret_cast<float*>(p.out) + ob;
-#pragma unroll
-                            for (int e = 0; e < T::EPL; e += 4)
-                                *reinterpret_cast<float4*>(dst + e) = make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]);
-                        } else {
-                            uint32_t w4[4];
-#pragma unroll
-                            for (int e = 0; e < T::EPL; e += 2) w4[e / 2] = pack_bf16(x[e], x[e + 1]);
-                            uint16_t* dst = reinterpret_cast<uint16_t*>(p.out) + ob;
-                            if constexpr (T::EPL == 8)
-                                *reinterpret_cast<uint4*>(dst) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-                            else
-                                *reinterpret_cast<uint2*>(dst) = make_uint2(w4[0], w4[1]);
-                        }
+                        store_out<T::EPL>(p, ob, x);
                     }
                 }
             }
@@ -708,9 +774,29 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const DecodePara
     }
 
     if (flags[0] && tid == 0) {
-        // a wait gave up: wait (bounded) for the copies still in flight before exiting
+        // a wait gave up: wait (bounded) for the copies still in flight
         for (int k = i_stop; k < issued; k++)
             (void)mbar_wait(smem_u32(&bars[k % NS]), (uint32_t)((k / NS) & 1));
+    }
+
+    // ---- merge the cut segments, spread over every CTA that holds a part
+    if (G > 1) {
+        if (!grid_barrier(p.barrier, (unsigned)G, &flags[2])) {
+            if (tid == 0) atomicOr(p.status, kStatusWaitTimeout);
+            return;
+        }
+        Cursor c0, c1;
+        cursor_locate(c0, w0, pref, B, HH);
+        cursor_locate(c1, w1 - 1, pref, B, HH);
+        for (int k = 0; k < 2; k++) {
+            const Cursor& c = k == 0 ? c0 : c1;
+            if (k == 1 && c1.b == c0.b && c1.hh == c0.hh) break;
+            const int64_t seg_w0 = (int64_t)pref[c.b] * HH + (int64_t)c.hh * c.npages;
+            if (seg_w0 >= w0 && seg_w0 + c.npages <= w1) continue;     // whole: already stored
+            const int i_first = owner_of(seg_w0, W, G);
+            const int i_last = owner_of(seg_w0 + c.npages - 1, W, G);
+            merge_segment<D>(p, c.b, c.hh / HB, c.hh % HB, seg_w0, i_first, i_last, W, G, fin);
+        }
     }
 }
 
@@ -768,6 +854,15 @@ cudaError_t plan_decode(const Layout& L, int B, int HB, int max_seq_len, DecodeP
     plan->stages = (int)stages;
     plan->threads = kDecThreads;
     plan->smem = (((size_t)stages * L.slab + 127) & ~(size_t)127) + fixed;
+    const void* kern = decode_kernel_for(L.fmt, L.D);
+    if (!kern) return cudaErrorInvalidValue;
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan->smem)) != cudaSuccess)
+        return e;
+    int resident = 0;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident, kern, kDecThreads, plan->smem)) != cudaSuccess)
+        return e;
+    if (resident < 1) return cudaErrorInvalidConfiguration;
+    if (resident < ctas) ctas = resident;
     const int64_t pages = (max_seq_len + L.P - 1) / L.P;
     int64_t work = (int64_t)B * pages * L.H * HB;
     int64_t grid = (int64_t)sms * ctas;
@@ -777,26 +872,29 @@ cudaError_t plan_decode(const Layout& L, int B, int HB, int max_seq_len, DecodeP
     return cudaSuccess;
 }
 
+static size_t partial_bytes(const Layout& L, int grid) {
+    return (((size_t)grid * 2 * (16 + 8 * (size_t)L.D) * sizeof(float)) + 255) & ~(size_t)255;
+}
+
 size_t decode_workspace_bytes(const Layout& L, int B, int HB, int grid) {
-    size_t partials = (size_t)grid * 2 * 8 * (L.D + 2) * sizeof(float);
-    size_t counters = (size_t)B * L.H * HB * sizeof(int);
-    return ((partials + 255) & ~(size_t)255) + ((counters + 255) & ~(size_t)255);
+    (void)B;
+    (void)HB;
+    return partial_bytes(L, grid) + 256;
 }
 
 void decode_workspace_zero_region(const Layout& L, int B, int HB, int grid, size_t* offset, size_t* bytes) {
-    size_t partials = (size_t)grid * 2 * 8 * (L.D + 2) * sizeof(float);
-    size_t counters = (size_t)B * L.H * HB * sizeof(int);
-    *offset = (partials + 255) & ~(size_t)255;
-    *bytes = (counters + 255) & ~(size_t)255;
+    (void)B;
+    (void)HB;
+    *offset = partial_bytes(L, grid);
+    *bytes = 256;
 }
 
 cudaError_t launch_decode(const DecodeParams& p, const DecodePlan& plan, cudaStream_t s) {
     const void* k = decode_kernel_for(p.L.fmt, p.L.D);
     if (!k) return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan.smem);
-    if (e != cudaSuccess) return e;
     void* args[] = {const_cast<DecodeParams*>(&p)};
-    return cudaLaunchKernel(k, dim3(plan.grid), dim3(plan.threads), args, plan.smem, s);
+    // cooperative: the merge after the grid barrier needs every CTA resident
+    return cudaLaunchCooperativeKernel(k, dim3(plan.grid), dim3(plan.threads), args, plan.smem, s);
 }
 
 }  // namespace kvq

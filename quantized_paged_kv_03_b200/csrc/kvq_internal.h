@@ -48,8 +48,8 @@ struct DecodeParams {
     float q_mult;                // softmax_scale * log2(e) * K tensor scale
     float o_mult;                // V tensor scale (1 otherwise)
     bool rot_k, rot_v;
-    float* partials;             // [gridDim.x][2][8 * (D + 2)]
-    int* counters;               // [B][H][HB], zero between calls
+    float* partials;             // [gridDim.x][2][16 + 8 * D]: (max, sum, output) of cut segments
+    unsigned* barrier;           // grid barrier: [0] arrivals (zero between calls), [1] generation
     uint32_t* status;
     int stages;                  // pipeline depth (page slabs in shared memory)
 };
