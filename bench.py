@@ -108,13 +108,13 @@ class ClockSampler:
 class Arm:
     """One workload on the GPU: cache with the prefix appended, step inputs in HBM."""
 
-    def __init__(self, cfg: int, fmt: str, seed_offset: int = 0):
+    def __init__(self, cfg: int, fmt: str, seed_offset: int = 0, batch: int | None = None):
         import torch
         import quantized_paged_kv_03_b200 as K
         self.torch, self.K = torch, K
         spec = I.CONFIGS[cfg]
         seed = I.SEED_BASE + cfg + 1000 * seed_offset
-        self.w = w = I.make_workload(cfg, fmt=fmt, seed=seed)
+        self.w = w = I.make_workload(cfg, fmt=fmt, seed=seed, B=batch)
         self.fmt = fmt
         self.tb = K.token_bytes(fmt, w.D)
         scales = None
@@ -327,6 +327,10 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--quick", action="store_true", help="headline workload only")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle baseline")
+    ap.add_argument("--config", type=int, default=HEADLINE_CONFIG,
+                    help="workload index for the headline line (profiling a single kernel)")
+    ap.add_argument("--format", default=None, help="format of that workload (default: its first)")
+    ap.add_argument("--batch", type=int, default=None, help="fewer sequences (small profiling case)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -344,21 +348,21 @@ def main():
     flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
     flush = lambda: flush_buf.fill_(1)
 
-    spec = I.CONFIGS[HEADLINE_CONFIG]
-    fmt = spec.formats[0]
-    arm = Arm(HEADLINE_CONFIG, fmt, seed_offset=rank)
+    spec = I.CONFIGS[args.config]
+    fmt = args.format or spec.formats[0]
+    arm = Arm(args.config, fmt, seed_offset=rank, batch=args.batch)
     clocks_path = os.path.join(ROOT, "gpurun_out", f"bench_clocks_r{rank}.csv")
     os.makedirs(os.path.dirname(clocks_path), exist_ok=True)
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(clocks_path) as clk:
-        t_wall = time.perf_counter()
-        app, dec = arm.run(args.steps, args.warmup, flush)
-        torch.cuda.synchronize()
-        if dist is not None:
-            dist.barrier()
-        t_wall = time.perf_counter() - t_wall
+    clk = ClockSampler(clocks_path).__enter__()     # sampled over every timed section below
+    t_wall = time.perf_counter()
+    app, dec = arm.run(args.steps, args.warmup, flush)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    t_wall = time.perf_counter() - t_wall
     step_ms = float((app + dec).mean())
     dec_ms = float(dec.mean())
     step_ms_max = max_over_ranks(step_ms, dist)
@@ -390,9 +394,11 @@ def main():
                 del a
                 torch.cuda.empty_cache()
 
+    clk.__exit__(None, None, None)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
-        cpu = oracle_sample(HEADLINE_CONFIG, fmt, budget_s=12.0)
+        cpu = oracle_sample(args.config, fmt, budget_s=12.0)
 
     if rank == 0:
         line = {

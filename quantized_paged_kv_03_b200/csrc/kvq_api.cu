@@ -195,6 +195,7 @@ int kvq_decode_attention(kvq_cache* cache, int32_t layer, const void* q, int32_t
     p.barrier = (unsigned*)((uint8_t*)workspace + zoff);
     p.status = (uint32_t*)cache->pool;
     p.stages = plan.stages;
+    p.pid_cap = plan.pid_cap;
     return cuda_status(launch_decode(p, plan, (cudaStream_t)stream));
 }
 

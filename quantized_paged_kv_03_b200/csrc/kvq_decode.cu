@@ -8,25 +8,27 @@
 // not arithmetic) make this a streaming kernel: its roofline is HBM bandwidth.
 //
 // Design (B200, sm_100a):
-//  * Persistent CTAs (4 warps).  The page-heads of the whole batch, ordered
-//    (sequence, kv-head, 8-head block, page), are cut into gridDim.x contiguous
-//    equal ranges, so ragged batches balance to within one page.
+//  * Persistent cooperative grid, 8 warps per CTA.  The page-heads of the whole
+//    batch, ordered (sequence, kv-head, 8-head block, page), are cut into
+//    gridDim.x contiguous equal ranges, so ragged batches balance to within
+//    one page.
 //  * Each page slab (K codes, K scales, V codes, V scales of one kv-head: one
 //    contiguous range in HBM) arrives with ONE cp.async.bulk into a shared-memory
-//    stage, completion tracked by an mbarrier; `stages` slabs are in flight.
-//  * Warp w takes 16-token tiles w, w+4, ... of each page.  Codes are turned
-//    into fp16 (exact for every format) in registers straight from shared
-//    memory and fed to mma.sync m16n8k16 with the GQA group (<= 8 query heads)
-//    as N: S^T = K q^T with tokens as M, then O^T += V^T P^T with head_dim as M
-//    (movmatrix transposes the V and P fragments).  Group scales are folded
-//    into fp32 S (K) or into P (V); NVFP4 scales go into the operand, where
-//    code x scale is exact in fp16.  q is split into hi + lo halves so the
-//    scores keep ~22 bits.
-//  * Online softmax in the log2 domain per warp; the four warps merge in
-//    shared memory at the end of each (sequence, kv-head) segment.  A segment
-//    cut by a CTA range boundary writes a partial (max, sum, unnormalised
-//    output) and the last CTA to finish that segment merges all partials
-//    (arrival counter in the workspace, reset by the merger): no second launch.
+//    stage, completion tracked by an mbarrier.  Warps release a stage with a
+//    shared counter; the last warp to release it issues the next copy into it,
+//    so warps never wait for each other page by page.
+//  * A 16-token tile is owned by a warp pair: each warp takes one half of
+//    head_dim.  Codes become fp16 (exact for every format) in registers straight
+//    from shared memory and feed mma.sync m16n8k16 with the GQA group (<= 8
+//    query heads) as N: S^T = K q^T (tokens as M, the pair adds its two halves
+//    through shared memory), then O^T += V^T P^T (head_dim as M; movmatrix
+//    transposes the V and P fragments).  Group scales are folded into fp32
+//    scores (K) or into P (V); NVFP4 scales go into the operand, where
+//    code x scale is exact in fp16.
+//  * Online softmax in the log2 domain; the warps merge in shared memory at
+//    the end of each (sequence, kv-head) segment.  A segment cut by a range
+//    boundary leaves a partial (max, sum, unnormalised output); after one grid
+//    barrier every CTA that holds a part merges a share of that segment.
 //  * Rotated K: q is rotated by the same normalised Hadamard-256 (orthonormal,
 //    so q.k is unchanged).  Rotated V: the output is rotated back (the matrix
 //    is symmetric and its own inverse).
@@ -34,9 +36,10 @@
 
 namespace kvq {
 
-constexpr int kDecThreads = 128;
+constexpr int kDecThreads = 256;   // 8 warps: 4 tile slots x 2 head_dim halves
 constexpr int kMaxStages = 8;
 constexpr int kMaxBatch = 4096;
+constexpr long kWaitPolls = 1l << 22;
 
 // ------------------------------------------------------------ PTX helpers
 
@@ -57,16 +60,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t phase) {
         : "memory");
     return ok != 0;
 }
-// Bounded wait: gives up after ~2^22 polls (each poll may suspend briefly).
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t phase) {
-    for (int i = 0; i < (1 << 22); i++)
+// Bounded wait for a stage.  Gives up after kWaitPolls polls, or at once when
+// another warp has already given up (`abort` set), so a failed copy never hangs
+// the CTA: every warp then runs through its remaining work without waiting.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t phase, volatile int* abort) {
+    for (long i = 0; i < kWaitPolls; i++) {
         if (mbar_try_wait(bar, phase)) return true;
+        if (*abort) return false;
+    }
+    *abort = 1;
     return false;
 }
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
                  "l"(src), "r"(bytes), "r"(bar)
                  : "memory");
+}
+__device__ __forceinline__ void pair_sync(int id) {   // the two warps of a tile pair
+    asm volatile("bar.sync %0, 64;" ::"r"(id) : "memory");
 }
 
 __device__ __forceinline__ void mma_f16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
@@ -100,15 +111,32 @@ __device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
     return r;
 }
 __device__ __forceinline__ uint32_t f16_splat(uint32_t h16) { return (h16 & 0xFFFFu) * 0x10001u; }
+// 2^x for x <= 0 (softmax weights): one MUFU instruction; results below 2^-126 flush to 0.
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Eight E2M1 codes (one word, element 2i in the low nibble of byte i) -> four
+// f16x2, byte i giving (element 2i, element 2i+1).  Exact.
+__device__ __forceinline__ void dec_e2m1x8(uint32_t w, uint32_t (&o)[4]) {
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\tmov.b32 {b0, b1, b2, b3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\tcvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\tcvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+        : "=r"(o[0]), "=r"(o[1]), "=r"(o[2]), "=r"(o[3])
+        : "r"(w));
+}
+// Four E4M3 codes (one word) -> two f16x2: (e0, e1), (e2, e3).  Exact.
+__device__ __forceinline__ void dec_e4m3x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
+    asm("{\n\t.reg .b16 h0, h1;\n\tmov.b32 {h0, h1}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, h0;\n\tcvt.rn.f16x2.e4m3x2 %1, h1;\n\t}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(w));
+}
 
 template <int NB>
-struct Bytes;   // NB bytes loaded from shared memory as 32-bit words
-template <>
-struct Bytes<8> { uint32_t w[2]; };
-template <>
-struct Bytes<16> { uint32_t w[4]; };
-template <>
-struct Bytes<32> { uint32_t w[8]; };
+struct Bytes { uint32_t w[NB / 4]; };   // NB bytes of one row, as words
 
 // Load NB (8/16/32) logical bytes at logical offset `lb` of a code row whose
 // 16-byte chunks are permuted by `swz`.
@@ -130,22 +158,26 @@ __device__ __forceinline__ Bytes<NB> lds_row(const uint8_t* row, int lb, int swz
     return b;
 }
 
-// Four consecutive codes e0..e3 of one row (element `4 * step` of a lane's
-// slice) -> f16x2 pairs (e0,e1) and (e2,e3), without any scale.
-template <int KIND, int NB>
-__device__ __forceinline__ void codes4_f16(const Bytes<NB>& b, int step, uint32_t& x01, uint32_t& x23) {
+// All codes of a lane's slice of one row -> f16x2 pairs: x[2*step] = elements
+// (4 step, 4 step + 1), x[2*step + 1] = (4 step + 2, 4 step + 3).  No scale.
+template <int KIND, int NB, int STEPS>
+__device__ __forceinline__ void slice_f16(const Bytes<NB>& b, uint32_t (&x)[2 * STEPS]) {
     if constexpr (kind_bits(KIND) == 16) {
-        x01 = b.w[2 * step];
-        x23 = b.w[2 * step + 1];
+#pragma unroll
+        for (int i = 0; i < 2 * STEPS; i++) x[i] = b.w[i];
     } else if constexpr (kind_bits(KIND) == 4) {
-        uint32_t h = (b.w[step >> 1] >> ((step & 1) * 16)) & 0xFFFFu;
-        x01 = dec_e2m1x2_f16x2(h & 0xFFu);
-        x23 = dec_e2m1x2_f16x2(h >> 8);
+#pragma unroll
+        for (int i = 0; i < STEPS / 2; i++) {
+            uint32_t o[4];
+            dec_e2m1x8(b.w[i], o);
+            x[4 * i] = o[0]; x[4 * i + 1] = o[1]; x[4 * i + 2] = o[2]; x[4 * i + 3] = o[3];
+        }
     } else if constexpr (KIND == RK_INT8_G64) {
-        dec_int8x4_f16x2(b.w[step], x01, x23);
+#pragma unroll
+        for (int i = 0; i < STEPS; i++) dec_int8x4_f16x2(b.w[i], x[2 * i], x[2 * i + 1]);
     } else {
-        x01 = dec_e4m3x2_f16x2(b.w[step] & 0xFFFFu);
-        x23 = dec_e4m3x2_f16x2(b.w[step] >> 16);
+#pragma unroll
+        for (int i = 0; i < STEPS; i++) dec_e4m3x4(b.w[i], x[2 * i], x[2 * i + 1]);
     }
 }
 
@@ -158,26 +190,36 @@ struct DecTraits {
     static constexpr int KCW = 16 * KCH, VCW = 16 * VCH;       // chunk widths in head_dim
     static constexpr int KNB = 4 * KCH * KBITS / 8;            // bytes per lane per K row load
     static constexpr int VNB = 4 * VCH * VBITS / 8;
+    static constexpr int KCHUNKS = KSTEPS / KCH, VCHUNKS = DTILES / VCH;
+    static constexpr int KC_HALF = KCHUNKS / 2, VC_HALF = VCHUNKS / 2;   // per warp of a pair
+    static constexpr int QS = (KK == RK_BF16RAW) ? 2 : 1;      // q split into hi (+ lo)
     static constexpr int EPL = D / 32;
+    static_assert(KCHUNKS % 2 == 0 && VCHUNKS % 2 == 0, "head_dim halves must hold whole chunks");
 };
 
 // Cursor over this CTA's page-heads: (sequence b, head pair hh = h*HB + hb, page).
 struct Cursor {
-    int b, hh, page, npages;
+    int b, hh, h, hb, page, npages;   // hh = h * HB + hb
 };
 
-__device__ __forceinline__ void cursor_next(Cursor& c, const int* pref, int B, int HH) {
+__device__ __forceinline__ void cursor_next(Cursor& c, const int* pref, int B, int HH, int HB) {
     if (++c.page < c.npages) return;
     c.page = 0;
-    if (++c.hh < HH) return;
-    c.hh = 0;
+    if (++c.hh < HH) {
+        if (++c.hb == HB) {
+            c.hb = 0;
+            c.h++;
+        }
+        return;
+    }
+    c.hh = c.h = c.hb = 0;
     do {
         c.b++;
     } while (c.b < B && pref[c.b + 1] == pref[c.b]);
     c.npages = (c.b < B) ? pref[c.b + 1] - pref[c.b] : 0;
 }
 
-__device__ __forceinline__ void cursor_locate(Cursor& c, int64_t w, const int* pref, int B, int HH) {
+__device__ __forceinline__ void cursor_locate(Cursor& c, int64_t w, const int* pref, int B, int HH, int HB) {
     int lo = 0, hi = B - 1;   // largest b with pref[b]*HH <= w
     while (lo < hi) {
         int mid = (lo + hi + 1) >> 1;
@@ -190,6 +232,8 @@ __device__ __forceinline__ void cursor_locate(Cursor& c, int64_t w, const int* p
     int64_t idx = w - (int64_t)pref[lo] * HH;
     c.hh = (int)(idx / c.npages);
     c.page = (int)(idx % c.npages);
+    c.h = c.hh / HB;
+    c.hb = c.hh % HB;
 }
 
 // CTA owning page-head w when W page-heads are cut into G equal ranges.
@@ -263,8 +307,9 @@ __device__ __forceinline__ void merge_segment(const DecodeParams& p, int b, int 
         const int64_t start = (int64_t)i * W / G;
         return p.partials + ((int64_t)i * 2 + (start >= seg_w0 ? 0 : 1)) * (16 + 8 * D);
     };
-    // segment max and sum per head: 16 lanes per head
-    {
+    // segment max and sum per head: 16 lanes per head (threads 0..127)
+    __syncthreads();
+    if (tid < 128) {
         const int g = tid >> 4, pl = tid & 15;
         float M = -INFINITY;
         for (int k = pl; k < P; k += 16) M = fmaxf(M, __ldcg(part_of(k) + g));
@@ -278,50 +323,56 @@ __device__ __forceinline__ void merge_segment(const DecodeParams& p, int b, int 
         }
 #pragma unroll
         for (int m = 1; m < 16; m <<= 1) L += __shfl_xor_sync(0xffffffffu, L, m);
-        __syncthreads();
         if (pl == 0) {
             fin[g] = M;
             fin[8 + g] = L;
         }
-        __syncthreads();
     }
+    __syncthreads();
     const int no = o1 - o0;
-    if (no <= 0) return;
-    int tpo = 1;
-    while (tpo < 16 && tpo * 2 * no <= kDecThreads) tpo *= 2;
-    const int per_pass = kDecThreads / tpo;
-    for (int ob = o0; ob < o1; ob += per_pass) {
-        const int o = ob + tid / tpo, pl = tid % tpo;
-        const bool valid = o < o1;
-        const int g = valid ? o / (D / 4) : 0, d4 = valid ? o % (D / 4) : 0;
-        const float M = fin[g];
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (valid) {
-            for (int k = pl; k < P; k += tpo) {
-                const float* pk = part_of(k);
-                const float mk = __ldcg(pk + g);
-                const float4 v = __ldcg(reinterpret_cast<const float4*>(pk + 16 + g * D) + d4);
-                const float wk = (mk == -INFINITY) ? 0.f : exp2f(mk - M);
-                acc.x = fmaf(wk, v.x, acc.x); acc.y = fmaf(wk, v.y, acc.y);
-                acc.z = fmaf(wk, v.z, acc.z); acc.w = fmaf(wk, v.w, acc.w);
+    if (no > 0) {
+        int tpo = 1;
+        while (tpo < 16 && tpo * 2 * no <= kDecThreads) tpo *= 2;
+        const int per_pass = kDecThreads / tpo;
+        for (int ob = o0; ob < o1; ob += per_pass) {
+            const int o = ob + tid / tpo, pl = tid % tpo;
+            const bool valid = o < o1;
+            const int g = valid ? o / (D / 4) : 0, d4 = valid ? o % (D / 4) : 0;
+            const float M = fin[g];
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (valid) {
+                for (int k = pl; k < P; k += tpo) {
+                    const float* pk = part_of(k);
+                    const float mk = __ldcg(pk + g);
+                    const float4 v = __ldcg(reinterpret_cast<const float4*>(pk + 16 + g * D) + d4);
+                    const float wk = (mk == -INFINITY) ? 0.f : exp2f(mk - M);
+                    acc.x = fmaf(wk, v.x, acc.x); acc.y = fmaf(wk, v.y, acc.y);
+                    acc.z = fmaf(wk, v.z, acc.z); acc.w = fmaf(wk, v.w, acc.w);
+                }
             }
-        }
-        for (int m = 1; m < tpo; m <<= 1) {
-            acc.x += __shfl_xor_sync(0xffffffffu, acc.x, m);
-            acc.y += __shfl_xor_sync(0xffffffffu, acc.y, m);
-            acc.z += __shfl_xor_sync(0xffffffffu, acc.z, m);
-            acc.w += __shfl_xor_sync(0xffffffffu, acc.w, m);
-        }
-        if (valid && pl == 0) {
-            const float Ls = fin[8 + g];
-            const float inv = (Ls > 0.f) ? p.o_mult / Ls : 0.f;
-            const float x[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
-            const int64_t oo = ((int64_t)b * p.Hq + h * p.G + hb * 8 + g) * D + 4 * d4;
-            store_out<4>(p, oo, x);
+            for (int m = 1; m < tpo; m <<= 1) {
+                acc.x += __shfl_xor_sync(0xffffffffu, acc.x, m);
+                acc.y += __shfl_xor_sync(0xffffffffu, acc.y, m);
+                acc.z += __shfl_xor_sync(0xffffffffu, acc.z, m);
+                acc.w += __shfl_xor_sync(0xffffffffu, acc.w, m);
+            }
+            if (valid && pl == 0) {
+                const float Ls = fin[8 + g];
+                const float inv = (Ls > 0.f) ? p.o_mult / Ls : 0.f;
+                const float x[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
+                const int64_t oo = ((int64_t)b * p.Hq + h * p.G + hb * 8 + g) * D + 4 * d4;
+                store_out<4>(p, oo, x);
+            }
         }
     }
     __syncthreads();
 }
+
+// Shared state of the stage producer (only the warp that issues a copy touches it).
+struct Producer {
+    Cursor c;
+    int issued;
+};
 
 template <int KK, int KV, int D>
 __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const DecodeParams p) {
@@ -329,23 +380,32 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const DecodePara
     extern __shared__ __align__(128) uint8_t smem[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int r = lane >> 2, j = lane & 3;
+    const int tw = warp & 3, hf = warp >> 2;     // tile slot, head_dim half
     const int H = p.L.H, P = p.L.P, HB = p.HB, HH = H * HB, B = p.B;
     const int64_t slab = p.L.slab;
     const int NS = p.stages;
 
     // shared memory carve-up
     size_t off = ((size_t)NS * slab + 127) & ~(size_t)127;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + off);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + off);   // full[stage]
     off += 8 * kMaxStages;
-    float* osm = reinterpret_cast<float*>(smem + off);   // [8][D]: q staging / output combine
-    off += 8 * D * 4;
-    float* wml = reinterpret_cast<float*>(smem + off);   // [4 warps][m 8, l 8]
+    int* rel = reinterpret_cast<int*>(smem + off);               // release count[stage]
+    off += 4 * kMaxStages;
+    Producer* prod = reinterpret_cast<Producer*>(smem + off);
+    off += 32;
+    float* osm = reinterpret_cast<float*>(smem + off);   // [8][D]: q staging / output combine / score exchange
+    off += (8 * D * 4 > 8192 ? 8 * D * 4 : 8192);
+    float4* xbuf = reinterpret_cast<float4*>(osm);       // [2 parity][4 tiles][2 halves][32 lanes]
+    float* wml = reinterpret_cast<float*>(smem + off);   // [4 tile warps][m 8, l 8]
     off += 4 * 16 * 4;
     float* fin = reinterpret_cast<float*>(smem + off);   // [m 8][l 8] of the merged segment
     off += 16 * 4;
-    int* flags = reinterpret_cast<int*>(smem + off);     // [0] abort, [1] last arriver
+    int* flags = reinterpret_cast<int*>(smem + off);     // [0] abort, [2] grid barrier ok
     off += 16;
     int* pref = reinterpret_cast<int*>(smem + off);      // [B + 1] page prefix
+    off += 4 * (size_t)(B + 1);
+    int* pids = reinterpret_cast<int*>(smem + off);      // [pid_cap] page ids of this CTA's range
+    volatile int* abort_flag = flags;
 
     // ---- page prefix over the batch (block scan)
     {
@@ -368,10 +428,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const DecodePara
             if (lane >= m) incl += v;
         }
         if (lane == 31) wml[warp] = __int_as_float(incl);
-        if (tid == 0) {
-            flags[0] = 0;
-            flags[1] = 0;
-        }
+        if (tid == 0) flags[0] = flags[1] = flags[2] = flags[3] = 0;
         __syncthreads();
         int base = 0;
         for (int w = 0; w < warp; w++) base += __float_as_int(wml[w]);
@@ -405,56 +462,67 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const DecodePara
     const int64_t w0 = (int64_t)blockIdx.x * W / G, w1 = (int64_t)(blockIdx.x + 1) * W / G;
     const int n = (int)(w1 - w0);
 
-    if (tid == 0) {
-        for (int s = 0; s < NS; s++) mbar_init(smem_u32(&bars[s]), 1);
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
-    __syncthreads();
-
-    // ---- producer: thread 0 keeps NS slabs in flight
-    Cursor pc{0, 0, 0, 0};
-    int issued = 0;
-    auto issue = [&](int s) {
-        int pid = p.block_table[(int64_t)pc.b * p.max_pages + pc.page];
+    // ---- page ids of this CTA's range, loaded in parallel up front so that a
+    // refill never waits on a block-table read
+    auto page_id = [&](int64_t w) {
+        Cursor c;
+        cursor_locate(c, w, pref, B, HH, HB);
+        int pid = p.block_table[(int64_t)c.b * p.max_pages + c.page];
         if (pid < 0 || pid >= p.L.num_pages) {
             atomicOr(p.status, kStatusBadPage);
             pid = 0;
         }
-        const uint8_t* src = p.slabs + ((int64_t)pid * H + pc.hh / HB) * slab;
+        return pid;
+    };
+    for (int k = tid; k < n && k < p.pid_cap; k += kDecThreads) pids[k] = page_id(w0 + k);
+    __syncthreads();
+
+    // ---- producer: the slab of the next page-head into a free stage
+    auto issue = [&](int s) {
+        Cursor& pc = prod->c;
+        const int k = prod->issued;
+        const int pid = (k < p.pid_cap) ? pids[k] : page_id(w0 + k);
+        const uint8_t* src = p.slabs + ((int64_t)pid * H + pc.h) * slab;
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         uint32_t bar = smem_u32(&bars[s]);
         mbar_expect_tx(bar, (uint32_t)slab);
         bulk_g2s(smem_u32(smem + (size_t)s * slab), src, (uint32_t)slab, bar);
+        cursor_next(pc, pref, B, HH, HB);
+        prod->issued++;
     };
     if (tid == 0) {
-        cursor_locate(pc, w0, pref, B, HH);
-        for (int s = 0; s < NS && issued < n; s++) {
-            issue(s);
-            cursor_next(pc, pref, B, HH);
-            issued++;
+        for (int s = 0; s < NS; s++) {
+            mbar_init(smem_u32(&bars[s]), 1);
+            rel[s] = 0;
         }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        cursor_locate(prod->c, w0, pref, B, HH, HB);
+        prod->issued = 0;
+        for (int s = 0; s < NS && s < n; s++) issue(s);
     }
+    __syncthreads();
 
-    // ---- consumer state
+    // ---- consumer state (warp pair: tile slot tw, head_dim half hf)
     Cursor cc;
-    cursor_locate(cc, w0, pref, B, HH);
-    uint32_t qh[T::KSTEPS][2], ql[T::KSTEPS][2];
-    float o[T::DTILES][4];
+    cursor_locate(cc, w0, pref, B, HH, HB);
+    const int tiles = P >> 4;    // 16-token tiles per page
+    int s = 0;                   // stage of page i
+    uint32_t ph = 0;             // mbarrier phase of that stage's current use
+    int seq_len = 0;
+    uint32_t qf[T::KSTEPS / 2][T::QS][2];
+    float o[T::DTILES / 2][4];
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
     bool seg_first = true;     // segment began at this CTA's first page
+    int xpar = 0;              // score-exchange buffer parity
 
-    int i_stop = n;
     for (int i = 0; i < n; i++) {
-        const int s = i % NS;
-        const bool seg_begin = (i == 0) || (cc.page == 0);
-        const int b = cc.b, h = cc.hh / HB, hb = cc.hh % HB;
-        if (seg_begin) {
+        const int b = cc.b, h = cc.h, hb = cc.hb;
+        if (i == 0 || cc.page == 0) {
+            // ---- segment start: q rows of this 8-head block, rotated and scaled
             seg_first = (i == 0);
-            // q rows of this 8-head block -> rotated, scaled fp32 in osm -> fragments
-#pragma unroll
-            for (int k = 0; k < 2; k++) {
-                const int nh = warp + 4 * k;
-                const int gq = hb * 8 + nh;
+            seq_len = p.seq_lens[b];
+            {
+                const int gq = hb * 8 + warp;   // warp w stages head w of the block
                 float x[8];
                 if (gq < p.G) {
                     const uint16_t* qrow = p.q + ((int64_t)b * p.Hq + h * p.G + gq) * D + lane * T::EPL;
@@ -470,107 +538,115 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const DecodePara
                     for (int e = 0; e < T::EPL; e++) x[e] = 0.f;
                 }
 #pragma unroll
-                for (int e = 0; e < T::EPL; e++) osm[nh * D + lane * T::EPL + e] = x[e];
+                for (int e = 0; e < T::EPL; e++) osm[warp * D + lane * T::EPL + e] = x[e];
             }
             __syncthreads();
 #pragma unroll
-            for (int st = 0; st < T::KSTEPS; st++) {
+            for (int sl = 0; sl < T::KSTEPS / 2; sl++) {
+                const int st = hf * (T::KSTEPS / 2) + sl;
                 const int c = st / T::KCH, ks = st % T::KCH;
                 const int d0 = T::KCW * c + 4 * T::KCH * j + 4 * ks;
                 const float* qr = osm + r * D + d0;
-                float v[4] = {qr[0], qr[1], qr[2], qr[3]};
-                float lo[4];
-                if constexpr (KK == RK_BF16RAW) {
+                const float v[4] = {qr[0], qr[1], qr[2], qr[3]};
+                if constexpr (T::QS == 2) {
+                    float lo[4];
 #pragma unroll
                     for (int e = 0; e < 4; e++) lo[e] = v[e] - __bfloat162float(__float2bfloat16_rn(v[e]));
-                    qh[st][0] = pack_bf16(v[0], v[1]);
-                    qh[st][1] = pack_bf16(v[2], v[3]);
-                    ql[st][0] = pack_bf16(lo[0], lo[1]);
-                    ql[st][1] = pack_bf16(lo[2], lo[3]);
+                    qf[sl][0][0] = pack_bf16(v[0], v[1]);
+                    qf[sl][0][1] = pack_bf16(v[2], v[3]);
+                    qf[sl][T::QS - 1][0] = pack_bf16(lo[0], lo[1]);
+                    qf[sl][T::QS - 1][1] = pack_bf16(lo[2], lo[3]);
                 } else {
-#pragma unroll
-                    for (int e = 0; e < 4; e++) lo[e] = v[e] - __half2float(__float2half_rn(v[e]));
-                    qh[st][0] = pack_f16(v[0], v[1]);
-                    qh[st][1] = pack_f16(v[2], v[3]);
-                    ql[st][0] = pack_f16(lo[0], lo[1]);
-                    ql[st][1] = pack_f16(lo[2], lo[3]);
+                    qf[sl][0][0] = pack_f16(v[0], v[1]);
+                    qf[sl][0][1] = pack_f16(v[2], v[3]);
                 }
             }
 #pragma unroll
-            for (int u = 0; u < T::DTILES; u++) o[u][0] = o[u][1] = o[u][2] = o[u][3] = 0.f;
+            for (int u = 0; u < T::DTILES / 2; u++) o[u][0] = o[u][1] = o[u][2] = o[u][3] = 0.f;
             m0 = m1 = -INFINITY;
             l0 = l1 = 0.f;
+            __syncthreads();   // osm becomes the score-exchange buffer
         }
 
         // wait for the slab
-        if (!mbar_wait(smem_u32(&bars[s]), (uint32_t)((i / NS) & 1))) {
-            atomicOr(p.status, kStatusWaitTimeout);
-            flags[0] = 1;
-        }
+        (void)mbar_wait(smem_u32(&bars[s]), ph, abort_flag);
 
-        // ---- compute: 16-token tiles of this page
+        // ---- this pair's 16-token tiles of the page
         const uint8_t* stg = smem + (size_t)s * slab;
         const uint8_t* kcodes = stg;
         const uint8_t* kscl = stg + p.L.off_ks;
         const uint8_t* vcodes = stg + p.L.off_vc;
         const uint8_t* vscl = stg + p.L.off_vs;
-        const int seq_len = p.seq_lens[b];
-        for (int mt = warp; mt < P / 16; mt += 4) {
+        for (int mt = tw; mt < tiles; mt += 4) {
             const int valid = seq_len - (cc.page * P + mt * 16);
-            if (valid <= 0) break;
+            if (valid <= 0) break;   // same decision in both warps of the pair
             const int ta = mt * 16 + r, tb = ta + 8;
-            // ---------- S^T = K q^T
+            // ---------- partial S^T = K q^T over this warp's half of head_dim
             float sc[4] = {0.f, 0.f, 0.f, 0.f};
-            const uint8_t* rowa = kcodes + (int64_t)ta * p.L.kc;
-            const uint8_t* rowb = kcodes + (int64_t)tb * p.L.kc;
-            const int swa = row_swizzle(KK, D, ta), swb = row_swizzle(KK, D, tb);
+            {
+                const uint8_t* rowa = kcodes + (int64_t)ta * p.L.kc;
+                const uint8_t* rowb = kcodes + (int64_t)tb * p.L.kc;
+                const int swa = row_swizzle(KK, D, ta), swb = row_swizzle(KK, D, tb);
 #pragma unroll
-            for (int c = 0; c < T::KSTEPS / T::KCH; c++) {
-                const int lb = (T::KCW * c + 4 * T::KCH * j) * T::KBITS / 8;
-                Bytes<T::KNB> ka = lds_row<T::KNB>(rowa, lb, swa);
-                Bytes<T::KNB> kb = lds_row<T::KNB>(rowb, lb, swb);
-                uint32_t sca = 0, scb = 0;
-                if constexpr (KK == RK_E2M1_G16) {
-                    const int g = (T::KCW * c + 16 * j) / 16;
-                    sca = f16_splat(dec_e4m3x2_f16x2(kscl[ta * p.L.ks + g]));
-                    scb = f16_splat(dec_e4m3x2_f16x2(kscl[tb * p.L.ks + g]));
-                }
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int ks = 0; ks < T::KCH; ks++) {
-                    const int st = c * T::KCH + ks;
-                    uint32_t a[4];
-                    codes4_f16<KK, T::KNB>(ka, ks, a[0], a[2]);
-                    codes4_f16<KK, T::KNB>(kb, ks, a[1], a[3]);
+                for (int cl = 0; cl < T::KC_HALF; cl++) {
+                    const int c = hf * T::KC_HALF + cl;
+                    const int lb = (T::KCW * c + 4 * T::KCH * j) * T::KBITS / 8;
+                    uint32_t xa[2 * T::KCH], xb[2 * T::KCH];
+                    slice_f16<KK, T::KNB, T::KCH>(lds_row<T::KNB>(rowa, lb, swa), xa);
+                    slice_f16<KK, T::KNB, T::KCH>(lds_row<T::KNB>(rowb, lb, swb), xb);
                     if constexpr (KK == RK_E2M1_G16) {
-                        a[0] = hmul2(a[0], sca); a[2] = hmul2(a[2], sca);
-                        a[1] = hmul2(a[1], scb); a[3] = hmul2(a[3], scb);
+                        const int g = (T::KCW * c + 16 * j) / 16;
+                        const uint32_t sa = f16_splat(dec_e4m3x2_f16x2(kscl[ta * p.L.ks + g]));
+                        const uint32_t sb = f16_splat(dec_e4m3x2_f16x2(kscl[tb * p.L.ks + g]));
+#pragma unroll
+                        for (int e = 0; e < 2 * T::KCH; e++) {
+                            xa[e] = hmul2(xa[e], sa);
+                            xb[e] = hmul2(xb[e], sb);
+                        }
                     }
-                    if constexpr (KK == RK_BF16RAW) {
-                        mma_bf16(acc, a, qh[st][0], qh[st][1]);
-                        mma_bf16(acc, a, ql[st][0], ql[st][1]);
+                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int ks = 0; ks < T::KCH; ks++) {
+                        const int sl = cl * T::KCH + ks;
+                        const uint32_t a[4] = {xa[2 * ks], xb[2 * ks], xa[2 * ks + 1], xb[2 * ks + 1]};
+#pragma unroll
+                        for (int qs = 0; qs < T::QS; qs++) {
+                            if constexpr (KK == RK_BF16RAW) mma_bf16(acc, a, qf[sl][qs][0], qf[sl][qs][1]);
+                            else mma_f16(acc, a, qf[sl][qs][0], qf[sl][qs][1]);
+                        }
+                    }
+                    if constexpr (KK == RK_INT8_G64 || KK == RK_E4M3_MX32) {
+                        float fa, fb;
+                        if constexpr (KK == RK_INT8_G64) {
+                            const uint16_t* s16 = reinterpret_cast<const uint16_t*>(kscl);
+                            fa = f16_bits_to_f32(s16[ta * (p.L.ks / 2) + c]);
+                            fb = f16_bits_to_f32(s16[tb * (p.L.ks / 2) + c]);
+                        } else {
+                            fa = ue8m0_to_f32(kscl[ta * p.L.ks + c]);
+                            fb = ue8m0_to_f32(kscl[tb * p.L.ks + c]);
+                        }
+                        sc[0] = fmaf(acc[0], fa, sc[0]);
+                        sc[1] = fmaf(acc[1], fa, sc[1]);
+                        sc[2] = fmaf(acc[2], fb, sc[2]);
+                        sc[3] = fmaf(acc[3], fb, sc[3]);
                     } else {
-                        mma_f16(acc, a, qh[st][0], qh[st][1]);
-                        mma_f16(acc, a, ql[st][0], ql[st][1]);
+                        sc[0] += acc[0]; sc[1] += acc[1]; sc[2] += acc[2]; sc[3] += acc[3];
                     }
                 }
-                if constexpr (KK == RK_INT8_G64 || KK == RK_E4M3_MX32) {
-                    float fa, fb;
-                    if constexpr (KK == RK_INT8_G64) {
-                        const uint16_t* s16 = reinterpret_cast<const uint16_t*>(kscl);
-                        fa = f16_bits_to_f32(s16[ta * (p.L.ks / 2) + c]);
-                        fb = f16_bits_to_f32(s16[tb * (p.L.ks / 2) + c]);
-                    } else {
-                        fa = ue8m0_to_f32(kscl[ta * p.L.ks + c]);
-                        fb = ue8m0_to_f32(kscl[tb * p.L.ks + c]);
-                    }
-                    sc[0] = fmaf(acc[0], fa, sc[0]);
-                    sc[1] = fmaf(acc[1], fa, sc[1]);
-                    sc[2] = fmaf(acc[2], fb, sc[2]);
-                    sc[3] = fmaf(acc[3], fb, sc[3]);
+            }
+            // ---------- add the two halves (same order in both warps: identical sums)
+            {
+                float4* mine = xbuf + ((xpar * 4 + tw) * 2 + hf) * 32 + lane;
+                const float4* other = xbuf + ((xpar * 4 + tw) * 2 + (hf ^ 1)) * 32 + lane;
+                *mine = make_float4(sc[0], sc[1], sc[2], sc[3]);
+                pair_sync(1 + tw);
+                const float4 ot = *other;
+                if (hf == 0) {
+                    sc[0] += ot.x; sc[1] += ot.y; sc[2] += ot.z; sc[3] += ot.w;
                 } else {
-                    sc[0] += acc[0]; sc[1] += acc[1]; sc[2] += acc[2]; sc[3] += acc[3];
+                    sc[0] = ot.x + sc[0]; sc[1] = ot.y + sc[1]; sc[2] = ot.z + sc[2]; sc[3] = ot.w + sc[3];
                 }
+                xpar ^= 1;
             }
             if constexpr (KK == RK_E4M3_ROW256) {
                 const uint16_t* s16 = reinterpret_cast<const uint16_t*>(kscl);
@@ -593,7 +669,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const DecodePara
                 const float a0 = (m0 == -INFINITY) ? 0.f : exp2f(m0 - n0);
                 const float a1 = (m1 == -INFINITY) ? 0.f : exp2f(m1 - n1);
 #pragma unroll
-                for (int u = 0; u < T::DTILES; u++) {
+                for (int u = 0; u < T::DTILES / 2; u++) {
                     o[u][0] *= a0; o[u][1] *= a1; o[u][2] *= a0; o[u][3] *= a1;
                 }
                 l0 *= a0;
@@ -602,12 +678,12 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const DecodePara
                 m1 = n1;
             }
             const float r0 = (m0 == -INFINITY) ? 0.f : m0, r1 = (m1 == -INFINITY) ? 0.f : m1;
-            const float p0 = exp2f(sc[0] - r0), p1 = exp2f(sc[1] - r1);
-            const float p2 = exp2f(sc[2] - r0), p3 = exp2f(sc[3] - r1);
+            const float p0 = fast_exp2(sc[0] - r0), p1 = fast_exp2(sc[1] - r1);
+            const float p2 = fast_exp2(sc[2] - r0), p3 = fast_exp2(sc[3] - r1);
             l0 += p0 + p2;
             l1 += p1 + p3;
 
-            // ---------- O^T += V^T P^T
+            // ---------- O^T += V^T P^T over this warp's half of head_dim
             // rows past seq_len hold bytes never written: keep them out of the
             // product entirely (their P is 0, but 0 x NaN would still be NaN)
             const bool oka = r < valid, okb = r + 8 < valid, partial = valid < 16;
@@ -626,7 +702,8 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const DecodePara
                 pb1 = movtrans(pack_f16(p2, p3));
             }
 #pragma unroll
-            for (int c = 0; c < T::DTILES / T::VCH; c++) {
+            for (int cl = 0; cl < T::VC_HALF; cl++) {
+                const int c = hf * T::VC_HALF + cl;
                 if constexpr (KV == RK_INT8_G64 || KV == RK_E4M3_MX32) {
                     float fa, fb;
                     if constexpr (KV == RK_INT8_G64) {
@@ -643,57 +720,62 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const DecodePara
                     pb1 = movtrans(pack_f16(p2 * fb, p3 * fb));
                 }
                 const int lb = (T::VCW * c + 4 * T::VCH * j) * T::VBITS / 8;
-                Bytes<T::VNB> va = lds_row<T::VNB>(vrowa, lb, vswa);
-                Bytes<T::VNB> vb = lds_row<T::VNB>(vrowb, lb, vswb);
-                uint32_t sva = 0, svb = 0;
+                uint32_t xa[2 * T::VCH], xb[2 * T::VCH];
+                slice_f16<KV, T::VNB, T::VCH>(lds_row<T::VNB>(vrowa, lb, vswa), xa);
+                slice_f16<KV, T::VNB, T::VCH>(lds_row<T::VNB>(vrowb, lb, vswb), xb);
                 if constexpr (KV == RK_E2M1_G16) {
                     const int g = (T::VCW * c + 16 * j) / 16;
-                    sva = f16_splat(dec_e4m3x2_f16x2(vscl[ta * p.L.vs + g]));
-                    svb = f16_splat(dec_e4m3x2_f16x2(vscl[tb * p.L.vs + g]));
+                    const uint32_t sa = f16_splat(dec_e4m3x2_f16x2(vscl[ta * p.L.vs + g]));
+                    const uint32_t sb = f16_splat(dec_e4m3x2_f16x2(vscl[tb * p.L.vs + g]));
+#pragma unroll
+                    for (int e = 0; e < 2 * T::VCH; e++) {
+                        xa[e] = hmul2(xa[e], sa);
+                        xb[e] = hmul2(xb[e], sb);
+                    }
+                }
+                if (partial) {
+#pragma unroll
+                    for (int e = 0; e < 2 * T::VCH; e++) {
+                        xa[e] = oka ? xa[e] : 0u;
+                        xb[e] = okb ? xb[e] : 0u;
+                    }
                 }
 #pragma unroll
                 for (int u = 0; u < T::VCH; u++) {
-                    uint32_t xa01, xa23, xb01, xb23;
-                    codes4_f16<KV, T::VNB>(va, u, xa01, xa23);
-                    codes4_f16<KV, T::VNB>(vb, u, xb01, xb23);
-                    if constexpr (KV == RK_E2M1_G16) {
-                        xa01 = hmul2(xa01, sva); xa23 = hmul2(xa23, sva);
-                        xb01 = hmul2(xb01, svb); xb23 = hmul2(xb23, svb);
-                    }
-                    if (partial) {
-                        if (!oka) xa01 = xa23 = 0u;
-                        if (!okb) xb01 = xb23 = 0u;
-                    }
-                    uint32_t a[4] = {movtrans(xa01), movtrans(xa23), movtrans(xb01), movtrans(xb23)};
-                    mma_f16(o[c * T::VCH + u], a, pb0, pb1);
+                    const uint32_t a[4] = {movtrans(xa[2 * u]), movtrans(xa[2 * u + 1]), movtrans(xb[2 * u]),
+                                           movtrans(xb[2 * u + 1])};
+                    mma_f16(o[cl * T::VCH + u], a, pb0, pb1);
                 }
             }
         }
 
-        const bool seg_end = (i == n - 1) || (cc.page == cc.npages - 1);
-        __syncthreads();   // every warp is done with stage s (and with osm)
-        if (flags[0]) {
-            i_stop = i + 1;
-            break;
-        }
-        if (tid == 0 && issued < n) {
-            issue(s);
-            cursor_next(pc, pref, B, HH);
-            issued++;
+        // ---- release stage s; the last warp to release it refills it
+        __syncwarp();
+        if (lane == 0) {
+            __threadfence_block();
+            const int old = atomicAdd(&rel[s], 1);
+            if (old == kDecThreads / 32 - 1) {
+                rel[s] = 0;
+                __threadfence_block();
+                if (prod->issued < n && !*abort_flag) issue(s);
+            }
         }
 
+        const bool seg_end = (i == n - 1) || (cc.page == cc.npages - 1);
         if (seg_end) {
-            // ---- merge the four warps: max, rescaled sums, rescaled outputs
+            // ---- merge the warps: max, rescaled sums, rescaled outputs.  The two
+            // warps of a pair hold the same (m, l); the half-0 warp reports them.
 #pragma unroll
             for (int m = 4; m < 32; m <<= 1) {
                 l0 += __shfl_xor_sync(0xffffffffu, l0, m);
                 l1 += __shfl_xor_sync(0xffffffffu, l1, m);
             }
-            if (r == 0) {
-                wml[warp * 16 + 2 * j] = m0;
-                wml[warp * 16 + 2 * j + 1] = m1;
-                wml[warp * 16 + 8 + 2 * j] = l0;
-                wml[warp * 16 + 8 + 2 * j + 1] = l1;
+            __syncthreads();   // all tiles of the segment done; osm free
+            if (hf == 0 && r == 0) {
+                wml[tw * 16 + 2 * j] = m0;
+                wml[tw * 16 + 2 * j + 1] = m1;
+                wml[tw * 16 + 8 + 2 * j] = l0;
+                wml[tw * 16 + 8 + 2 * j + 1] = l1;
             }
             __syncthreads();
             float M0 = -INFINITY, M1 = -INFINITY;
@@ -715,9 +797,10 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const DecodePara
                 fin[8 + tid] = Ls;
             }
             for (int w = 0; w < 4; w++) {
-                if (warp == w) {
+                if (tw == w) {   // both halves write disjoint head_dim ranges
 #pragma unroll
-                    for (int u = 0; u < T::DTILES; u++) {
+                    for (int ul = 0; ul < T::DTILES / 2; ul++) {
+                        const int u = hf * (T::DTILES / 2) + ul;
                         const int c = u / T::VCH, uu = u % T::VCH;
                         const int base = T::VCW * c + 4 * uu;
                         const int da = base + 4 * T::VCH * (r >> 1) + (r & 1);   // logical row r
@@ -725,11 +808,11 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const DecodePara
                         float* oa0 = osm + (2 * j) * D;
                         float* oa1 = osm + (2 * j + 1) * D;
                         if (w == 0) {
-                            oa0[da] = o[u][0] * f0; oa1[da] = o[u][1] * f1;
-                            oa0[db] = o[u][2] * f0; oa1[db] = o[u][3] * f1;
+                            oa0[da] = o[ul][0] * f0; oa1[da] = o[ul][1] * f1;
+                            oa0[db] = o[ul][2] * f0; oa1[db] = o[ul][3] * f1;
                         } else {
-                            oa0[da] += o[u][0] * f0; oa1[da] += o[u][1] * f1;
-                            oa0[db] += o[u][2] * f0; oa1[db] += o[u][3] * f1;
+                            oa0[da] += o[ul][0] * f0; oa1[da] += o[ul][1] * f1;
+                            oa0[db] += o[ul][2] * f0; oa1[db] += o[ul][3] * f1;
                         }
                     }
                 }
@@ -744,9 +827,8 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const DecodePara
             const bool whole = (seg_w0 >= w0) && (seg_w0 + cc.npages <= w1);
             float* part = p.partials + ((int64_t)blockIdx.x * 2 + (seg_first ? 0 : 1)) * (16 + 8 * D);
             if (!whole && tid < 16) part[tid] = fin[tid];
-#pragma unroll
-            for (int k = 0; k < 2; k++) {
-                const int nh = warp + 4 * k;
+            {
+                const int nh = warp;   // warp w finishes head w of the block
                 const int gq = hb * 8 + nh;
                 if (gq < p.G) {
                     const float Ls = fin[8 + nh];
@@ -770,13 +852,24 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const DecodePara
             }
             __syncthreads();   // osm and fin are free again
         }
-        cursor_next(cc, pref, B, HH);
+        cursor_next(cc, pref, B, HH, HB);
+        if (++s == NS) {
+            s = 0;
+            ph ^= 1u;
+        }
     }
 
-    if (flags[0] && tid == 0) {
-        // a wait gave up: wait (bounded) for the copies still in flight
-        for (int k = i_stop; k < issued; k++)
-            (void)mbar_wait(smem_u32(&bars[k % NS]), (uint32_t)((k / NS) & 1));
+    __syncthreads();
+    if (*abort_flag) {
+        if (tid == 0) {
+            atomicOr(p.status, kStatusWaitTimeout);
+            // wait (bounded) for the copies still in flight: the last NS issued
+            int dummy = 0;
+            const int k0 = prod->issued > NS ? prod->issued - NS : 0;
+            for (int k = k0; k < prod->issued; k++)
+                (void)mbar_wait(smem_u32(&bars[k % NS]), (uint32_t)((k / NS) & 1), &dummy);
+        }
+        __syncthreads();
     }
 
     // ---- merge the cut segments, spread over every CTA that holds a part
@@ -786,8 +879,8 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const DecodePara
             return;
         }
         Cursor c0, c1;
-        cursor_locate(c0, w0, pref, B, HH);
-        cursor_locate(c1, w1 - 1, pref, B, HH);
+        cursor_locate(c0, w0, pref, B, HH, HB);
+        cursor_locate(c1, w1 - 1, pref, B, HH, HB);
         for (int k = 0; k < 2; k++) {
             const Cursor& c = k == 0 ? c0 : c1;
             if (k == 1 && c1.b == c0.b && c1.hh == c0.hh) break;
@@ -795,7 +888,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const DecodePara
             if (seg_w0 >= w0 && seg_w0 + c.npages <= w1) continue;     // whole: already stored
             const int i_first = owner_of(seg_w0, W, G);
             const int i_last = owner_of(seg_w0 + c.npages - 1, W, G);
-            merge_segment<D>(p, c.b, c.hh / HB, c.hh % HB, seg_w0, i_first, i_last, W, G, fin);
+            merge_segment<D>(p, c.b, c.h, c.hb, seg_w0, i_first, i_last, W, G, fin);
         }
     }
 }
@@ -830,8 +923,10 @@ bool decode_supported(int fmt, int D) {
     return D == 128 || D == 256;
 }
 
-static size_t fixed_smem(int D, int B) {
-    return 8 * kMaxStages + 8 * (size_t)D * 4 + 4 * 16 * 4 + 16 * 4 + 16 + 4 * (size_t)(B + 1) + 128;
+static size_t fixed_smem(int D, int B, int pid_cap) {
+    const size_t osm = 8 * (size_t)D * 4 > 8192 ? 8 * (size_t)D * 4 : 8192;
+    return 8 * kMaxStages + 4 * kMaxStages + 32 + osm + 4 * 16 * 4 + 16 * 4 + 16 + 4 * (size_t)(B + 1) +
+           4 * (size_t)pid_cap + 128;
 }
 
 cudaError_t plan_decode(const Layout& L, int B, int HB, int max_seq_len, DecodePlan* plan) {
@@ -842,34 +937,35 @@ cudaError_t plan_decode(const Layout& L, int B, int HB, int max_seq_len, DecodeP
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&smem_blk, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess) return e;
-    const size_t fixed = fixed_smem(L.D, B);
-    int ctas = 2;
-    int64_t stages = ((int64_t)smem_sm / 2 - 1024 - (int64_t)fixed) / L.slab;
-    if (stages < 3) {
-        ctas = 1;
-        stages = ((int64_t)smem_blk - (int64_t)fixed) / L.slab;
-    }
-    if (stages < 2) return cudaErrorInvalidValue;
-    if (stages > 6) stages = 6;
-    plan->stages = (int)stages;
-    plan->threads = kDecThreads;
-    plan->smem = (((size_t)stages * L.slab + 127) & ~(size_t)127) + fixed;
     const void* kern = decode_kernel_for(L.fmt, L.D);
     if (!kern) return cudaErrorInvalidValue;
-    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan->smem)) != cudaSuccess)
-        return e;
-    int resident = 0;
-    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident, kern, kDecThreads, plan->smem)) != cudaSuccess)
-        return e;
-    if (resident < 1) return cudaErrorInvalidConfiguration;
-    if (resident < ctas) ctas = resident;
     const int64_t pages = (max_seq_len + L.P - 1) / L.P;
-    int64_t work = (int64_t)B * pages * L.H * HB;
-    int64_t grid = (int64_t)sms * ctas;
-    if (work < grid) grid = work;
-    if (grid < 1) grid = 1;
-    plan->grid = (int)grid;
-    return cudaSuccess;
+    const int64_t work = (int64_t)B * pages * L.H * HB > 0 ? (int64_t)B * pages * L.H * HB : 1;
+    // two CTAs per SM when three stages fit, else one CTA with a deeper pipeline
+    for (int ctas = 2; ctas >= 1; ctas--) {
+        const int64_t grid = (int64_t)sms * ctas < work ? (int64_t)sms * ctas : work;
+        int64_t cap = (work + grid - 1) / grid + 1;
+        if (cap > 4096) cap = 4096;
+        const size_t fixed = fixed_smem(L.D, B, (int)cap);
+        const int64_t budget = ctas == 2 ? (int64_t)smem_sm / 2 - 1024 : (int64_t)smem_blk;
+        int64_t stages = (budget - (int64_t)fixed) / L.slab;
+        if (stages > 6) stages = 6;
+        if (stages < (ctas == 2 ? 3 : 2)) continue;
+        const size_t smem = (((size_t)stages * L.slab + 127) & ~(size_t)127) + fixed;
+        if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+            return e;
+        int resident = 0;
+        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident, kern, kDecThreads, smem)) != cudaSuccess)
+            return e;
+        if (resident < ctas) continue;
+        plan->stages = (int)stages;
+        plan->threads = kDecThreads;
+        plan->pid_cap = (int)cap;
+        plan->smem = smem;
+        plan->grid = (int)grid;
+        return cudaSuccess;
+    }
+    return cudaErrorInvalidConfiguration;
 }
 
 static size_t partial_bytes(const Layout& L, int grid) {

@@ -52,6 +52,7 @@ struct DecodeParams {
     unsigned* barrier;           // grid barrier: [0] arrivals (zero between calls), [1] generation
     uint32_t* status;
     int stages;                  // pipeline depth (page slabs in shared memory)
+    int pid_cap;                 // page ids of a CTA's range preloaded into shared memory
 };
 
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
@@ -61,7 +62,7 @@ cudaError_t launch_encode(int code, const float* x, int64_t n, uint8_t* out, cud
 
 // Decode: grid / smem plan for a layout (host side), then the launch.
 struct DecodePlan {
-    int grid, stages, threads;
+    int grid, stages, threads, pid_cap;
     size_t smem;
 };
 cudaError_t plan_decode(const Layout& L, int B, int HB, int max_seq_len, DecodePlan* plan);
