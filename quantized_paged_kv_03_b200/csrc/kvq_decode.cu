@@ -138,20 +138,22 @@ __device__ __forceinline__ void dec_e4m3x4(uint32_t w, uint32_t& lo, uint32_t& h
 template <int NB>
 struct Bytes { uint32_t w[NB / 4]; };   // NB bytes of one row, as words
 
-// Load NB (8/16/32) logical bytes at logical offset `lb` of a code row whose
-// 16-byte chunks are permuted by `swz`.
+// Load NB (8/16/32) bytes of a code row at byte offset `off` from `base`
+// (base 32-byte aligned, off 8- or 16-byte aligned).  A 32-byte slice is two
+// 16-byte chunks c, c+1 with c even; the row permutation of 16-bit rows flips
+// bit 0 of the chunk index, so the second chunk sits at off ^ 16.
 template <int NB>
-__device__ __forceinline__ Bytes<NB> lds_row(const uint8_t* row, int lb, int swz) {
+__device__ __forceinline__ Bytes<NB> lds_bytes(const uint8_t* base, uint32_t off) {
     Bytes<NB> b;
     if constexpr (NB == 8) {
-        uint2 v = *reinterpret_cast<const uint2*>(row + phys_byte(lb, swz));
+        uint2 v = *reinterpret_cast<const uint2*>(base + off);
         b.w[0] = v.x; b.w[1] = v.y;
     } else if constexpr (NB == 16) {
-        uint4 v = *reinterpret_cast<const uint4*>(row + phys_byte(lb, swz));
+        uint4 v = *reinterpret_cast<const uint4*>(base + off);
         b.w[0] = v.x; b.w[1] = v.y; b.w[2] = v.z; b.w[3] = v.w;
     } else {
-        uint4 v0 = *reinterpret_cast<const uint4*>(row + phys_byte(lb, swz));
-        uint4 v1 = *reinterpret_cast<const uint4*>(row + phys_byte(lb + 16, swz));
+        uint4 v0 = *reinterpret_cast<const uint4*>(base + off);
+        uint4 v1 = *reinterpret_cast<const uint4*>(base + (off ^ 16u));
         b.w[0] = v0.x; b.w[1] = v0.y; b.w[2] = v0.z; b.w[3] = v0.w;
         b.w[4] = v1.x; b.w[5] = v1.y; b.w[6] = v1.z; b.w[7] = v1.w;
     }
@@ -193,6 +195,8 @@ struct DecTraits {
     static constexpr int KCHUNKS = KSTEPS / KCH, VCHUNKS = DTILES / VCH;
     static constexpr int KC_HALF = KCHUNKS / 2, VC_HALF = VCHUNKS / 2;   // per warp of a pair
     static constexpr int QS = (KK == RK_BF16RAW) ? 2 : 1;      // q split into hi (+ lo)
+    static constexpr int KC = row_code_bytes(KK, D), KS = row_scale_bytes(KK, D);   // row bytes
+    static constexpr int VC = row_code_bytes(KV, D), VS = row_scale_bytes(KV, D);
     static constexpr int EPL = D / 32;
     static_assert(KCHUNKS % 2 == 0 && VCHUNKS % 2 == 0, "head_dim halves must hold whole chunks");
 };
@@ -515,6 +519,33 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const DecodePara
     bool seg_first = true;     // segment began at this CTA's first page
     int xpar = 0;              // score-exchange buffer parity
 
+    // Per-lane byte offsets inside a stage, fixed for the whole kernel: lane
+    // (r, j) reads token rows r and r + 8 of a tile (same chunk permutation, since
+    // the permutation depends on the row modulo 4) at the chunks of its half.
+    const int swk = row_swizzle(KK, D, r), swv = row_swizzle(KV, D, r);
+    uint32_t koff[T::KC_HALF], voff[T::VC_HALF], ksoff[T::KC_HALF], vsoff[T::VC_HALF];
+#pragma unroll
+    for (int cl = 0; cl < T::KC_HALF; cl++) {
+        const int c = hf * T::KC_HALF + cl;
+        koff[cl] = r * T::KC + phys_byte((T::KCW * c + 4 * T::KCH * j) * T::KBITS / 8, swk);
+        if constexpr (KK == RK_E2M1_G16) ksoff[cl] = r * T::KS + (T::KCW * c + 16 * j) / 16;
+        else if constexpr (KK == RK_INT8_G64) ksoff[cl] = r * T::KS + 2 * c;
+        else if constexpr (KK == RK_E4M3_MX32) ksoff[cl] = r * T::KS + c;
+        else ksoff[cl] = r * T::KS;
+    }
+#pragma unroll
+    for (int cl = 0; cl < T::VC_HALF; cl++) {
+        const int c = hf * T::VC_HALF + cl;
+        voff[cl] = r * T::VC + phys_byte((T::VCW * c + 4 * T::VCH * j) * T::VBITS / 8, swv);
+        if constexpr (KV == RK_E2M1_G16) vsoff[cl] = r * T::VS + (T::VCW * c + 16 * j) / 16;
+        else if constexpr (KV == RK_INT8_G64) vsoff[cl] = r * T::VS + 2 * c;
+        else if constexpr (KV == RK_E4M3_MX32) vsoff[cl] = r * T::VS + c;
+        else vsoff[cl] = r * T::VS;
+    }
+    const uint32_t off_ks = (uint32_t)p.L.off_ks, off_vc = (uint32_t)p.L.off_vc, off_vs = (uint32_t)p.L.off_vs;
+    float4* xmine = xbuf + (tw * 2 + hf) * 32 + lane;          // parity 0; parity 1 is +8*32
+    const float4* xother = xbuf + (tw * 2 + (hf ^ 1)) * 32 + lane;
+
     for (int i = 0; i < n; i++) {
         const int b = cc.b, h = cc.h, hb = cc.hb;
         if (i == 0 || cc.page == 0) {
@@ -572,75 +603,61 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const DecodePara
         (void)mbar_wait(smem_u32(&bars[s]), ph, abort_flag);
 
         // ---- this pair's 16-token tiles of the page
-        const uint8_t* stg = smem + (size_t)s * slab;
-        const uint8_t* kcodes = stg;
-        const uint8_t* kscl = stg + p.L.off_ks;
-        const uint8_t* vcodes = stg + p.L.off_vc;
-        const uint8_t* vscl = stg + p.L.off_vs;
+        const uint32_t stg = (uint32_t)s * (uint32_t)slab;   // byte offset of the stage
         for (int mt = tw; mt < tiles; mt += 4) {
             const int valid = seq_len - (cc.page * P + mt * 16);
             if (valid <= 0) break;   // same decision in both warps of the pair
-            const int ta = mt * 16 + r, tb = ta + 8;
+            const uint32_t kt = stg + mt * 16 * T::KC, kst = stg + off_ks + mt * 16 * T::KS;
+            const uint32_t vt = stg + off_vc + mt * 16 * T::VC, vst = stg + off_vs + mt * 16 * T::VS;
             // ---------- partial S^T = K q^T over this warp's half of head_dim
             float sc[4] = {0.f, 0.f, 0.f, 0.f};
-            {
-                const uint8_t* rowa = kcodes + (int64_t)ta * p.L.kc;
-                const uint8_t* rowb = kcodes + (int64_t)tb * p.L.kc;
-                const int swa = row_swizzle(KK, D, ta), swb = row_swizzle(KK, D, tb);
 #pragma unroll
-                for (int cl = 0; cl < T::KC_HALF; cl++) {
-                    const int c = hf * T::KC_HALF + cl;
-                    const int lb = (T::KCW * c + 4 * T::KCH * j) * T::KBITS / 8;
-                    uint32_t xa[2 * T::KCH], xb[2 * T::KCH];
-                    slice_f16<KK, T::KNB, T::KCH>(lds_row<T::KNB>(rowa, lb, swa), xa);
-                    slice_f16<KK, T::KNB, T::KCH>(lds_row<T::KNB>(rowb, lb, swb), xb);
-                    if constexpr (KK == RK_E2M1_G16) {
-                        const int g = (T::KCW * c + 16 * j) / 16;
-                        const uint32_t sa = f16_splat(dec_e4m3x2_f16x2(kscl[ta * p.L.ks + g]));
-                        const uint32_t sb = f16_splat(dec_e4m3x2_f16x2(kscl[tb * p.L.ks + g]));
+            for (int cl = 0; cl < T::KC_HALF; cl++) {
+                uint32_t xa[2 * T::KCH], xb[2 * T::KCH];
+                slice_f16<KK, T::KNB, T::KCH>(lds_bytes<T::KNB>(smem + kt, koff[cl]), xa);
+                slice_f16<KK, T::KNB, T::KCH>(lds_bytes<T::KNB>(smem + kt, koff[cl] + 8 * T::KC), xb);
+                if constexpr (KK == RK_E2M1_G16) {
+                    const uint32_t sa = f16_splat(dec_e4m3x2_f16x2(smem[kst + ksoff[cl]]));
+                    const uint32_t sb = f16_splat(dec_e4m3x2_f16x2(smem[kst + ksoff[cl] + 8 * T::KS]));
 #pragma unroll
-                        for (int e = 0; e < 2 * T::KCH; e++) {
-                            xa[e] = hmul2(xa[e], sa);
-                            xb[e] = hmul2(xb[e], sb);
-                        }
+                    for (int e = 0; e < 2 * T::KCH; e++) {
+                        xa[e] = hmul2(xa[e], sa);
+                        xb[e] = hmul2(xb[e], sb);
                     }
-                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                }
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                    for (int ks = 0; ks < T::KCH; ks++) {
-                        const int sl = cl * T::KCH + ks;
-                        const uint32_t a[4] = {xa[2 * ks], xb[2 * ks], xa[2 * ks + 1], xb[2 * ks + 1]};
+                for (int ks = 0; ks < T::KCH; ks++) {
+                    const int sl = cl * T::KCH + ks;
+                    const uint32_t a[4] = {xa[2 * ks], xb[2 * ks], xa[2 * ks + 1], xb[2 * ks + 1]};
 #pragma unroll
-                        for (int qs = 0; qs < T::QS; qs++) {
-                            if constexpr (KK == RK_BF16RAW) mma_bf16(acc, a, qf[sl][qs][0], qf[sl][qs][1]);
-                            else mma_f16(acc, a, qf[sl][qs][0], qf[sl][qs][1]);
-                        }
+                    for (int qs = 0; qs < T::QS; qs++) {
+                        if constexpr (KK == RK_BF16RAW) mma_bf16(acc, a, qf[sl][qs][0], qf[sl][qs][1]);
+                        else mma_f16(acc, a, qf[sl][qs][0], qf[sl][qs][1]);
                     }
-                    if constexpr (KK == RK_INT8_G64 || KK == RK_E4M3_MX32) {
-                        float fa, fb;
-                        if constexpr (KK == RK_INT8_G64) {
-                            const uint16_t* s16 = reinterpret_cast<const uint16_t*>(kscl);
-                            fa = f16_bits_to_f32(s16[ta * (p.L.ks / 2) + c]);
-                            fb = f16_bits_to_f32(s16[tb * (p.L.ks / 2) + c]);
-                        } else {
-                            fa = ue8m0_to_f32(kscl[ta * p.L.ks + c]);
-                            fb = ue8m0_to_f32(kscl[tb * p.L.ks + c]);
-                        }
-                        sc[0] = fmaf(acc[0], fa, sc[0]);
-                        sc[1] = fmaf(acc[1], fa, sc[1]);
-                        sc[2] = fmaf(acc[2], fb, sc[2]);
-                        sc[3] = fmaf(acc[3], fb, sc[3]);
+                }
+                if constexpr (KK == RK_INT8_G64 || KK == RK_E4M3_MX32) {
+                    float fa, fb;
+                    if constexpr (KK == RK_INT8_G64) {
+                        fa = f16_bits_to_f32(*reinterpret_cast<const uint16_t*>(smem + kst + ksoff[cl]));
+                        fb = f16_bits_to_f32(*reinterpret_cast<const uint16_t*>(smem + kst + ksoff[cl] + 8 * T::KS));
                     } else {
-                        sc[0] += acc[0]; sc[1] += acc[1]; sc[2] += acc[2]; sc[3] += acc[3];
+                        fa = ue8m0_to_f32(smem[kst + ksoff[cl]]);
+                        fb = ue8m0_to_f32(smem[kst + ksoff[cl] + 8 * T::KS]);
                     }
+                    sc[0] = fmaf(acc[0], fa, sc[0]);
+                    sc[1] = fmaf(acc[1], fa, sc[1]);
+                    sc[2] = fmaf(acc[2], fb, sc[2]);
+                    sc[3] = fmaf(acc[3], fb, sc[3]);
+                } else {
+                    sc[0] += acc[0]; sc[1] += acc[1]; sc[2] += acc[2]; sc[3] += acc[3];
                 }
             }
             // ---------- add the two halves (same order in both warps: identical sums)
             {
-                float4* mine = xbuf + ((xpar * 4 + tw) * 2 + hf) * 32 + lane;
-                const float4* other = xbuf + ((xpar * 4 + tw) * 2 + (hf ^ 1)) * 32 + lane;
-                *mine = make_float4(sc[0], sc[1], sc[2], sc[3]);
+                *(xmine + xpar * 256) = make_float4(sc[0], sc[1], sc[2], sc[3]);
                 pair_sync(1 + tw);
-                const float4 ot = *other;
+                const float4 ot = *(xother + xpar * 256);
                 if (hf == 0) {
                     sc[0] += ot.x; sc[1] += ot.y; sc[2] += ot.z; sc[3] += ot.w;
                 } else {
@@ -649,33 +666,39 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const DecodePara
                 xpar ^= 1;
             }
             if constexpr (KK == RK_E4M3_ROW256) {
-                const uint16_t* s16 = reinterpret_cast<const uint16_t*>(kscl);
-                const float fa = f16_bits_to_f32(s16[ta * (p.L.ks / 2)]);
-                const float fb = f16_bits_to_f32(s16[tb * (p.L.ks / 2)]);
+                const float fa = f16_bits_to_f32(*reinterpret_cast<const uint16_t*>(smem + kst + ksoff[0]));
+                const float fb = f16_bits_to_f32(*reinterpret_cast<const uint16_t*>(smem + kst + ksoff[0] + 8 * T::KS));
                 sc[0] *= fa; sc[1] *= fa; sc[2] *= fb; sc[3] *= fb;
             }
-            if (r >= valid) sc[0] = sc[1] = -INFINITY;
-            if (r + 8 >= valid) sc[2] = sc[3] = -INFINITY;
+            const bool oka = r < valid, okb = r + 8 < valid;
+            if (!oka) sc[0] = sc[1] = -INFINITY;
+            if (!okb) sc[2] = sc[3] = -INFINITY;
 
-            // ---------- online softmax (log2 domain), heads 2j and 2j+1
-            float x0 = fmaxf(sc[0], sc[2]), x1 = fmaxf(sc[1], sc[3]);
+            // ---------- online softmax (log2 domain), heads 2j and 2j+1.  The
+            // running max is raised (with a warp-wide reduction and a rescale of
+            // the accumulators) only when a score exceeds it by more than 2^3;
+            // otherwise weights up to 8 are kept as they are.
+            {
+                const float x0 = fmaxf(sc[0], sc[2]), x1 = fmaxf(sc[1], sc[3]);
+                if (__any_sync(0xffffffffu, (x0 > m0 + 3.f) || (x1 > m1 + 3.f))) {
+                    float y0 = x0, y1 = x1;
 #pragma unroll
-            for (int m = 4; m < 32; m <<= 1) {
-                x0 = fmaxf(x0, __shfl_xor_sync(0xffffffffu, x0, m));
-                x1 = fmaxf(x1, __shfl_xor_sync(0xffffffffu, x1, m));
-            }
-            const float n0 = fmaxf(m0, x0), n1 = fmaxf(m1, x1);
-            if (__any_sync(0xffffffffu, (n0 > m0) || (n1 > m1))) {
-                const float a0 = (m0 == -INFINITY) ? 0.f : exp2f(m0 - n0);
-                const float a1 = (m1 == -INFINITY) ? 0.f : exp2f(m1 - n1);
+                    for (int m = 4; m < 32; m <<= 1) {
+                        y0 = fmaxf(y0, __shfl_xor_sync(0xffffffffu, y0, m));
+                        y1 = fmaxf(y1, __shfl_xor_sync(0xffffffffu, y1, m));
+                    }
+                    const float n0 = fmaxf(m0, y0), n1 = fmaxf(m1, y1);
+                    const float a0 = (m0 == -INFINITY) ? 0.f : fast_exp2(m0 - n0);
+                    const float a1 = (m1 == -INFINITY) ? 0.f : fast_exp2(m1 - n1);
 #pragma unroll
-                for (int u = 0; u < T::DTILES / 2; u++) {
-                    o[u][0] *= a0; o[u][1] *= a1; o[u][2] *= a0; o[u][3] *= a1;
+                    for (int u = 0; u < T::DTILES / 2; u++) {
+                        o[u][0] *= a0; o[u][1] *= a1; o[u][2] *= a0; o[u][3] *= a1;
+                    }
+                    l0 *= a0;
+                    l1 *= a1;
+                    m0 = n0;
+                    m1 = n1;
                 }
-                l0 *= a0;
-                l1 *= a1;
-                m0 = n0;
-                m1 = n1;
             }
             const float r0 = (m0 == -INFINITY) ? 0.f : m0, r1 = (m1 == -INFINITY) ? 0.f : m1;
             const float p0 = fast_exp2(sc[0] - r0), p1 = fast_exp2(sc[1] - r1);
@@ -686,15 +709,11 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const DecodePara
             // ---------- O^T += V^T P^T over this warp's half of head_dim
             // rows past seq_len hold bytes never written: keep them out of the
             // product entirely (their P is 0, but 0 x NaN would still be NaN)
-            const bool oka = r < valid, okb = r + 8 < valid, partial = valid < 16;
-            const uint8_t* vrowa = vcodes + (int64_t)ta * p.L.vc;
-            const uint8_t* vrowb = vcodes + (int64_t)tb * p.L.vc;
-            const int vswa = row_swizzle(KV, D, ta), vswb = row_swizzle(KV, D, tb);
+            const bool partial = valid < 16;
             uint32_t pb0 = 0, pb1 = 0;   // P'^T fragment (B operand)
             if constexpr (KV == RK_E4M3_ROW256) {
-                const uint16_t* s16 = reinterpret_cast<const uint16_t*>(vscl);
-                const float fa = oka ? f16_bits_to_f32(s16[ta * (p.L.vs / 2)]) : 0.f;
-                const float fb = okb ? f16_bits_to_f32(s16[tb * (p.L.vs / 2)]) : 0.f;
+                const float fa = oka ? f16_bits_to_f32(*reinterpret_cast<const uint16_t*>(smem + vst + vsoff[0])) : 0.f;
+                const float fb = okb ? f16_bits_to_f32(*reinterpret_cast<const uint16_t*>(smem + vst + vsoff[0] + 8 * T::VS)) : 0.f;
                 pb0 = movtrans(pack_f16(p0 * fa, p1 * fa));
                 pb1 = movtrans(pack_f16(p2 * fb, p3 * fb));
             } else if constexpr (KV != RK_INT8_G64 && KV != RK_E4M3_MX32) {
@@ -703,30 +722,26 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const DecodePara
             }
 #pragma unroll
             for (int cl = 0; cl < T::VC_HALF; cl++) {
-                const int c = hf * T::VC_HALF + cl;
                 if constexpr (KV == RK_INT8_G64 || KV == RK_E4M3_MX32) {
                     float fa, fb;
                     if constexpr (KV == RK_INT8_G64) {
-                        const uint16_t* s16 = reinterpret_cast<const uint16_t*>(vscl);
-                        fa = f16_bits_to_f32(s16[ta * (p.L.vs / 2) + c]);
-                        fb = f16_bits_to_f32(s16[tb * (p.L.vs / 2) + c]);
+                        fa = f16_bits_to_f32(*reinterpret_cast<const uint16_t*>(smem + vst + vsoff[cl]));
+                        fb = f16_bits_to_f32(*reinterpret_cast<const uint16_t*>(smem + vst + vsoff[cl] + 8 * T::VS));
                     } else {
-                        fa = ue8m0_to_f32(vscl[ta * p.L.vs + c]);
-                        fb = ue8m0_to_f32(vscl[tb * p.L.vs + c]);
+                        fa = ue8m0_to_f32(smem[vst + vsoff[cl]]);
+                        fb = ue8m0_to_f32(smem[vst + vsoff[cl] + 8 * T::VS]);
                     }
                     fa = oka ? fa : 0.f;
                     fb = okb ? fb : 0.f;
                     pb0 = movtrans(pack_f16(p0 * fa, p1 * fa));
                     pb1 = movtrans(pack_f16(p2 * fb, p3 * fb));
                 }
-                const int lb = (T::VCW * c + 4 * T::VCH * j) * T::VBITS / 8;
                 uint32_t xa[2 * T::VCH], xb[2 * T::VCH];
-                slice_f16<KV, T::VNB, T::VCH>(lds_row<T::VNB>(vrowa, lb, vswa), xa);
-                slice_f16<KV, T::VNB, T::VCH>(lds_row<T::VNB>(vrowb, lb, vswb), xb);
+                slice_f16<KV, T::VNB, T::VCH>(lds_bytes<T::VNB>(smem + vt, voff[cl]), xa);
+                slice_f16<KV, T::VNB, T::VCH>(lds_bytes<T::VNB>(smem + vt, voff[cl] + 8 * T::VC), xb);
                 if constexpr (KV == RK_E2M1_G16) {
-                    const int g = (T::VCW * c + 16 * j) / 16;
-                    const uint32_t sa = f16_splat(dec_e4m3x2_f16x2(vscl[ta * p.L.vs + g]));
-                    const uint32_t sb = f16_splat(dec_e4m3x2_f16x2(vscl[tb * p.L.vs + g]));
+                    const uint32_t sa = f16_splat(dec_e4m3x2_f16x2(smem[vst + vsoff[cl]]));
+                    const uint32_t sb = f16_splat(dec_e4m3x2_f16x2(smem[vst + vsoff[cl] + 8 * T::VS]));
 #pragma unroll
                     for (int e = 0; e < 2 * T::VCH; e++) {
                         xa[e] = hmul2(xa[e], sa);
