@@ -275,22 +275,30 @@ def dist_setup(n):
     return rank, world, dist
 
 
-def max_over_ranks(x: float, dist) -> float:
+def max_over_ranks(x: float, dist, device="cuda") -> float:
     if dist is None:
         return x
     import torch
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
 
-def sum_over_ranks(x: float, dist) -> float:
+def sum_over_ranks(x: float, dist, device="cuda") -> float:
     if dist is None:
         return x
     import torch
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.SUM)
     return float(t.item())
+
+
+def whole_job_rate(units_this_rank: float, ms_this_rank: float, dist, device="cuda"):
+    """Units processed by all ranks / the slowest rank's time (per second), and
+    that time: each rank runs its own replica (weak scaling)."""
+    ms = max_over_ranks(ms_this_rank, dist, device)
+    total = sum_over_ranks(units_this_rank, dist, device)
+    return total / (ms * 1e-3), ms
 
 
 def reference_arm(args):
@@ -365,12 +373,12 @@ def main():
     t_wall = time.perf_counter() - t_wall
     step_ms = float((app + dec).mean())
     dec_ms = float(dec.mean())
-    step_ms_max = max_over_ranks(step_ms, dist)
-    dec_ms_max = max_over_ranks(dec_ms, dist)
     step_bytes = arm.dec_bytes + arm.app_bytes
+    bytes_per_s, step_ms_max = whole_job_rate(step_bytes, step_ms, dist)
+    value = bytes_per_s / 1e9
+    tokens, _ = whole_job_rate(arm.w.B, step_ms, dist)
+    dec_ms_max = max_over_ranks(dec_ms, dist)
     total_bytes = sum_over_ranks(step_bytes, dist)
-    value = total_bytes / (step_ms_max * 1e-3) / 1e9
-    tokens = sum_over_ranks(arm.w.B, dist) / (step_ms_max * 1e-3)
 
     e2e_ts, h2d, d2h = arm.run_e2e(max(5, args.steps // 2), args.warmup, flush)
     e2e_ms = max_over_ranks(float(e2e_ts.mean()), dist)
