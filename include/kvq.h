@@ -149,6 +149,23 @@ int kvq_decode_attention(kvq_cache* cache, int32_t layer, const void* q, int32_t
                          void* out, int32_t out_fp32, float softmax_scale,
                          void* workspace, size_t workspace_bytes, void* stream);
 
+/* One decode step in one launch: append every sequence's newest token and
+ * attend.  Equivalent to kvq_append of token seq_len[b] - 1 of each sequence
+ * (at the slot block_table[b][(seq_len[b]-1) / page_size] * page_size +
+ * (seq_len[b]-1) % page_size) followed by kvq_decode_attention with the same
+ * arguments, but the new rows are quantised inside the decode kernel: the CTA
+ * that reads a sequence's last page quantises the new token into its on-chip
+ * copy of that page and into the cache ([NInfer]: every decoded token re-reads
+ * the whole KV, so a step should not pay a second launch for its one new row).
+ *   k_new, v_new  bf16 [batch][n_kv_heads][head_dim], 16-byte aligned; rows of
+ *                 sequences with seq_len 0 are ignored.
+ * All other arguments, results and errors as kvq_decode_attention. */
+int kvq_append_decode(kvq_cache* cache, int32_t layer, const void* k_new, const void* v_new,
+                      const void* q, int32_t n_q_heads, const int32_t* block_table,
+                      int32_t max_pages_per_seq, const int32_t* seq_lens, int32_t batch,
+                      int32_t max_seq_len, void* out, int32_t out_fp32, float softmax_scale,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
 /* Size of the fixed device scratch array used by kvq_decode_attention_noalloc. */
 #define KVQ_NOALLOC_SCRATCH_BYTES (8u << 20)
 

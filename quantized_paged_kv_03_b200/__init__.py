@@ -62,6 +62,8 @@ def lib() -> ctypes.CDLL:
         "kvq_decode_workspace_bytes": (sz, [P, i32, i32, i32]),
         "kvq_decode_attention": (ctypes.c_int, [P, i32, P, i32, P, i32, P, i32, i32, P, i32, f32,
                                                 P, sz, P]),
+        "kvq_append_decode": (ctypes.c_int, [P, i32, P, P, P, i32, P, i32, P, i32, i32, P, i32, f32,
+                                             P, sz, P]),
         "kvq_decode_attention_noalloc": (ctypes.c_int, [P, i32, P, i32, P, i32, P, i32, i32, P, i32,
                                                         f32, P]),
         "kvq_dequant": (ctypes.c_int, [P, i32, P, i32, P, P, P]),
@@ -82,7 +84,7 @@ def lib() -> ctypes.CDLL:
 def exported_symbols():
     return ["kvq_token_bytes", "kvq_row_bytes", "kvq_cache_bytes", "kvq_cache_create",
             "kvq_cache_destroy", "kvq_append", "kvq_decode_workspace_bytes",
-            "kvq_decode_attention", "kvq_decode_attention_noalloc", "kvq_dequant", "kvq_read_rows", "kvq_encode",
+            "kvq_decode_attention", "kvq_append_decode", "kvq_decode_attention_noalloc", "kvq_dequant", "kvq_read_rows", "kvq_encode",
             "kvq_read_device_status", "kvq_status_string", "kvq_version"]
 
 
@@ -240,6 +242,33 @@ class KVCache:
                                           _ptr(out), int(out_fp32), float(softmax_scale),
                                           _ptr(ws), ws.numel(), _stream(stream)),
                "decode_attention")
+        return out
+
+    def append_decode(self, layer: int, k_new, v_new, q, block_table, seq_lens, max_seq_len: int,
+                      out=None, out_fp32: bool = True, softmax_scale: float = 0.0, workspace=None,
+                      stream=None):
+        """One decode step in one launch: append token seq_len[b] - 1 of every
+        sequence (k_new, v_new: bf16 [B, H_kv, D]) and attend over [0, seq_len)."""
+        import torch
+        _dev_tensor(k_new, torch.bfloat16, "k_new")
+        _dev_tensor(v_new, torch.bfloat16, "v_new")
+        _dev_tensor(q, torch.bfloat16, "q")
+        _dev_tensor(block_table, torch.int32, "block_table")
+        _dev_tensor(seq_lens, torch.int32, "seq_lens")
+        B, Hq, D = q.shape
+        if k_new.numel() != B * self.n_kv_heads * D or v_new.numel() != k_new.numel():
+            raise KVQError("append_decode: k_new/v_new must be [B, H_kv, D]")
+        if out is None:
+            out = torch.empty((B, Hq, D), dtype=torch.float32 if out_fp32 else torch.bfloat16,
+                              device=q.device)
+        else:
+            _dev_tensor(out, torch.float32 if out_fp32 else torch.bfloat16, "out")
+        ws = self.workspace(B, Hq, max_seq_len) if workspace is None else workspace
+        _check(lib().kvq_append_decode(self._h, layer, _ptr(k_new), _ptr(v_new), _ptr(q), Hq,
+                                       _ptr(block_table), block_table.shape[1], _ptr(seq_lens), B,
+                                       max_seq_len, _ptr(out), int(out_fp32), float(softmax_scale),
+                                       _ptr(ws), ws.numel(), _stream(stream)),
+               "append_decode")
         return out
 
     def decode_attention_noalloc(self, layer: int, q, block_table, seq_lens, max_seq_len: int, out,

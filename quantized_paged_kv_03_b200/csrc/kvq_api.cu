@@ -154,10 +154,32 @@ size_t kvq_decode_workspace_bytes(const kvq_cache* cache, int32_t batch, int32_t
     return decode_workspace_bytes(cache->L, batch, HB, plan.grid);
 }
 
+static int decode_common(kvq_cache* cache, int32_t layer, const void* k_new, const void* v_new, const void* q,
+                         int32_t n_q_heads, const int32_t* block_table, int32_t max_pages_per_seq,
+                         const int32_t* seq_lens, int32_t batch, int32_t max_seq_len, void* out, int32_t out_fp32,
+                         float softmax_scale, void* workspace, size_t workspace_bytes, void* stream);
+
 int kvq_decode_attention(kvq_cache* cache, int32_t layer, const void* q, int32_t n_q_heads, const int32_t* block_table,
                          int32_t max_pages_per_seq, const int32_t* seq_lens, int32_t batch, int32_t max_seq_len,
                          void* out, int32_t out_fp32, float softmax_scale, void* workspace, size_t workspace_bytes,
                          void* stream) {
+    return decode_common(cache, layer, nullptr, nullptr, q, n_q_heads, block_table, max_pages_per_seq, seq_lens,
+                         batch, max_seq_len, out, out_fp32, softmax_scale, workspace, workspace_bytes, stream);
+}
+
+int kvq_append_decode(kvq_cache* cache, int32_t layer, const void* k_new, const void* v_new, const void* q,
+                      int32_t n_q_heads, const int32_t* block_table, int32_t max_pages_per_seq,
+                      const int32_t* seq_lens, int32_t batch, int32_t max_seq_len, void* out, int32_t out_fp32,
+                      float softmax_scale, void* workspace, size_t workspace_bytes, void* stream) {
+    if (batch > 0 && (!k_new || !v_new || ((uintptr_t)k_new & 15) || ((uintptr_t)v_new & 15))) return KVQ_ERR_ARG;
+    return decode_common(cache, layer, k_new, v_new, q, n_q_heads, block_table, max_pages_per_seq, seq_lens, batch,
+                         max_seq_len, out, out_fp32, softmax_scale, workspace, workspace_bytes, stream);
+}
+
+static int decode_common(kvq_cache* cache, int32_t layer, const void* k_new, const void* v_new, const void* q,
+                         int32_t n_q_heads, const int32_t* block_table, int32_t max_pages_per_seq,
+                         const int32_t* seq_lens, int32_t batch, int32_t max_seq_len, void* out, int32_t out_fp32,
+                         float softmax_scale, void* workspace, size_t workspace_bytes, void* stream) {
     int G, HB;
     int st = decode_shape(cache, batch, n_q_heads, max_seq_len, &G, &HB);
     if (st != KVQ_OK) return st;
@@ -196,6 +218,10 @@ int kvq_decode_attention(kvq_cache* cache, int32_t layer, const void* q, int32_t
     p.status = (uint32_t*)cache->pool;
     p.stages = plan.stages;
     p.pid_cap = plan.pid_cap;
+    p.k_new = (const uint16_t*)k_new;
+    p.v_new = (const uint16_t*)v_new;
+    p.k_scale = cache->tensor_scales[2 * layer];
+    p.v_scale = cache->tensor_scales[2 * layer + 1];
     return cuda_status(launch_decode(p, plan, (cudaStream_t)stream));
 }
 

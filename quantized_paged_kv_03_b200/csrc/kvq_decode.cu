@@ -32,7 +32,7 @@
 //  * Rotated K: q is rotated by the same normalised Hadamard-256 (orthonormal,
 //    so q.k is unchanged).  Rotated V: the output is rotated back (the matrix
 //    is symmetric and its own inverse).
-#include "kvq_internal.h"
+#include "kvq_quant.cuh"
 
 namespace kvq {
 
@@ -604,6 +604,32 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const DecodePara
 
         // ---- this pair's 16-token tiles of the page
         const uint32_t stg = (uint32_t)s * (uint32_t)slab;   // byte offset of the stage
+
+        if (p.k_new != nullptr && cc.page == cc.npages - 1) {
+            // fused append: the sequence's newest token (position seq_len - 1) lies
+            // in its last page.  Quantise it into this stage, over whatever the copy
+            // brought, and into the cache (one head block writes the cache).
+            const int t = (seq_len - 1) - cc.page * P;
+            if (warp < 2) {
+                const int pid = (i < p.pid_cap) ? pids[i] : page_id(w0 + i);
+                uint8_t* g = p.slabs + ((int64_t)pid * H + h) * slab;
+                uint8_t* st = smem + stg;
+                if (warp == 0) {
+                    const uint16_t* src = p.k_new + ((int64_t)b * H + h) * D;
+                    quantize_row<KK, D>(src, p.rot_k, p.k_scale, st + t * T::KC, st + off_ks + t * T::KS, t, lane);
+                    if (hb == 0)
+                        quantize_row<KK, D>(src, p.rot_k, p.k_scale, g + t * T::KC, g + off_ks + t * T::KS, t, lane);
+                } else {
+                    const uint16_t* src = p.v_new + ((int64_t)b * H + h) * D;
+                    quantize_row<KV, D>(src, p.rot_v, p.v_scale, st + off_vc + t * T::VC, st + off_vs + t * T::VS,
+                                        t, lane);
+                    if (hb == 0)
+                        quantize_row<KV, D>(src, p.rot_v, p.v_scale, g + off_vc + t * T::VC, g + off_vs + t * T::VS,
+                                            t, lane);
+                }
+            }
+            asm volatile("bar.sync 5, %0;" ::"r"(kDecThreads) : "memory");
+        }
         for (int mt = tw; mt < tiles; mt += 4) {
             const int valid = seq_len - (cc.page * P + mt * 16);
             if (valid <= 0) break;   // same decision in both warps of the pair

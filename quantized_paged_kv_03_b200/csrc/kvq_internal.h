@@ -36,7 +36,7 @@ struct DequantParams {
 
 struct DecodeParams {
     Layout L;
-    const uint8_t* slabs;        // first slab of the layer
+    uint8_t* slabs;              // first slab of the layer (written only by the fused append)
     const uint16_t* q;           // bf16 [B][Hq][D]
     int Hq, G, HB;               // query heads, GQA group, 8-head blocks per kv-head
     const int32_t* block_table;
@@ -53,6 +53,9 @@ struct DecodeParams {
     uint32_t* status;
     int stages;                  // pipeline depth (page slabs in shared memory)
     int pid_cap;                 // page ids of a CTA's range preloaded into shared memory
+    const uint16_t* k_new;       // fused append: bf16 [B][H][D] rows of each sequence's newest
+    const uint16_t* v_new;       //   token (position seq_len - 1), or null for decode only
+    float k_scale, v_scale;      // per-tensor scales of the append (FP8_TENSOR)
 };
 
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s);

@@ -116,3 +116,41 @@ def test_decode_many_sequences_balanced_split():
     want = oc.decode(w.q, w.block_table, w.seq_lens, threads=8)
     ratio, err = attn_errors(got, want, w)
     assert ratio <= 1.0, err
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("fmt,cfg,D,P,lengths,H,Hq", [
+    ("int8_g64", 1, 256, 64, [1, 64, 65, 700, 1100], 2, 8),
+    ("nvfp4_g16", 2, 256, 64, [333, 900], 2, 12),
+    ("k8v4", 3, 256, 64, [2000, 129], 2, 12),
+    ("mxfp8_g32", 4, 128, 128, [600, 128, 1], 2, 16),
+    ("fp8_tensor", 4, 128, 64, [512, 77], 2, 16),
+    ("bf16", 4, 128, 64, [300, 2], 2, 16)])
+def test_fused_append_decode_equals_append_then_decode(fmt, cfg, D, P, lengths, H, Hq):
+    """kvq_append_decode stores the same codes as kvq_append and returns the
+    same output as kvq_decode_attention run after it."""
+    w = workload(cfg, D, P, lengths, H, Hq, seed=13)
+    scales = tensor_scales(w) if fmt == "fp8_tensor" else (1.0, 1.0)
+    sc = scales if fmt == "fp8_tensor" else None
+    kp, vp, sp = w.prefix()
+    kn, vn, sn = w.new_tokens()
+    ref = gpu_cache(w, fmt, 0, sc)
+    fused = gpu_cache(w, fmt, 0, sc)
+    for c in (ref, fused):
+        c.append(0, bf16_dev(kp), bf16_dev(vp), dev(sp))
+    ref.append(0, bf16_dev(kn), bf16_dev(vn), dev(sn))
+    want = gpu_decode(ref, w)
+    q, bt, sl = bf16_dev(w.q), dev(w.block_table), dev(w.seq_lens)
+    got = fused.append_decode(0, bf16_dev(kn), bf16_dev(vn), q, bt, sl, w.max_seq_len)
+    torch.cuda.synchronize()
+    assert np.array_equal(got.cpu().numpy().astype(np.float64), want)
+    for a, b in zip(ref.read_rows(0, dev(sn)), fused.read_rows(0, dev(sn))):
+        assert torch.equal(a, b)
+    # and against the oracle
+    oc = oracle_cache(w, fmt, 0, scales)
+    oc.append(kp, vp, sp)
+    oc.append(kn, vn, sn)
+    ratio, err = attn_errors(got.cpu().numpy().astype(np.float64),
+                             oc.decode(w.q, w.block_table, w.seq_lens, threads=8), w)
+    assert ratio <= 1.0, err
+    assert fused.read_device_status() == 0
