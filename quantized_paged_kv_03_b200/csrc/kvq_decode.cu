@@ -400,6 +400,8 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const DecodePara
     float* osm = reinterpret_cast<float*>(smem + off);   // [8][D]: q staging / output combine / score exchange
     off += (8 * D * 4 > 8192 ? 8 * D * 4 : 8192);
     float4* xbuf = reinterpret_cast<float4*>(osm);       // [2 parity][4 tiles][2 halves][32 lanes]
+    uint8_t* qst = smem + off;                           // q fragments of the segment (fp16 / bf16 hi, lo)
+    off += 8 * (size_t)D * 2 * T::QS;
     float* wml = reinterpret_cast<float*>(smem + off);   // [4 tile warps][m 8, l 8]
     off += 4 * 16 * 4;
     float* fin = reinterpret_cast<float*>(smem + off);   // [m 8][l 8] of the merged segment
@@ -553,12 +555,23 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const DecodePara
             seg_first = (i == 0);
             seq_len = p.seq_lens[b];
             {
-                const int gq = hb * 8 + warp;   // warp w stages head w of the block
+                // warp w stages head w of the block, already in the MMA fragment
+                // order: for k-step st, lane group j, head n, the 4 values of that
+                // lane's slice as fp16 pairs (hi, and lo for a bf16 split)
+                const int gq = hb * 8 + warp;
                 float x[8];
                 if (gq < p.G) {
                     const uint16_t* qrow = p.q + ((int64_t)b * p.Hq + h * p.G + gq) * D + lane * T::EPL;
+                    uint32_t raw[4];
+                    if constexpr (T::EPL == 8) {
+                        const uint4 v = *reinterpret_cast<const uint4*>(qrow);
+                        raw[0] = v.x; raw[1] = v.y; raw[2] = v.z; raw[3] = v.w;
+                    } else {
+                        const uint2 v = *reinterpret_cast<const uint2*>(qrow);
+                        raw[0] = v.x; raw[1] = v.y; raw[2] = raw[3] = 0;
+                    }
 #pragma unroll
-                    for (int e = 0; e < T::EPL; e++) x[e] = bf16_bits_to_f32(qrow[e]);
+                    for (int e = 0; e < T::EPL; e++) x[e] = bf16_bits_to_f32((raw[e >> 1] >> ((e & 1) * 16)) & 0xFFFFu);
                     if constexpr (D == 256) {
                         if (p.rot_k) fwht256_warp(x, lane);
                     }
@@ -569,34 +582,41 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const DecodePara
                     for (int e = 0; e < T::EPL; e++) x[e] = 0.f;
                 }
 #pragma unroll
-                for (int e = 0; e < T::EPL; e++) osm[warp * D + lane * T::EPL + e] = x[e];
+                for (int g4 = 0; g4 < T::EPL / 4; g4++) {
+                    const int d0 = lane * T::EPL + 4 * g4;
+                    const int c = d0 / T::KCW, rem = d0 % T::KCW;
+                    const int jj = rem / (4 * T::KCH), ks = (rem % (4 * T::KCH)) / 4;
+                    const int st = c * T::KCH + ks;
+                    const float* v = x + 4 * g4;
+                    const int slot = (st * 4 + jj) * 8 + warp;
+                    if constexpr (T::QS == 2) {
+                        float lo[4];
+#pragma unroll
+                        for (int e = 0; e < 4; e++) lo[e] = v[e] - __bfloat162float(__float2bfloat16_rn(v[e]));
+                        reinterpret_cast<uint4*>(qst)[slot] = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]),
+                                                                         pack_bf16(lo[0], lo[1]), pack_bf16(lo[2], lo[3]));
+                    } else {
+                        reinterpret_cast<uint2*>(qst)[slot] = make_uint2(pack_f16(v[0], v[1]), pack_f16(v[2], v[3]));
+                    }
+                }
             }
             __syncthreads();
 #pragma unroll
             for (int sl = 0; sl < T::KSTEPS / 2; sl++) {
-                const int st = hf * (T::KSTEPS / 2) + sl;
-                const int c = st / T::KCH, ks = st % T::KCH;
-                const int d0 = T::KCW * c + 4 * T::KCH * j + 4 * ks;
-                const float* qr = osm + r * D + d0;
-                const float v[4] = {qr[0], qr[1], qr[2], qr[3]};
+                const int slot = ((hf * (T::KSTEPS / 2) + sl) * 4 + j) * 8 + r;
                 if constexpr (T::QS == 2) {
-                    float lo[4];
-#pragma unroll
-                    for (int e = 0; e < 4; e++) lo[e] = v[e] - __bfloat162float(__float2bfloat16_rn(v[e]));
-                    qf[sl][0][0] = pack_bf16(v[0], v[1]);
-                    qf[sl][0][1] = pack_bf16(v[2], v[3]);
-                    qf[sl][T::QS - 1][0] = pack_bf16(lo[0], lo[1]);
-                    qf[sl][T::QS - 1][1] = pack_bf16(lo[2], lo[3]);
+                    const uint4 v = reinterpret_cast<const uint4*>(qst)[slot];
+                    qf[sl][0][0] = v.x; qf[sl][0][1] = v.y;
+                    qf[sl][T::QS - 1][0] = v.z; qf[sl][T::QS - 1][1] = v.w;
                 } else {
-                    qf[sl][0][0] = pack_f16(v[0], v[1]);
-                    qf[sl][0][1] = pack_f16(v[2], v[3]);
+                    const uint2 v = reinterpret_cast<const uint2*>(qst)[slot];
+                    qf[sl][0][0] = v.x; qf[sl][0][1] = v.y;
                 }
             }
 #pragma unroll
             for (int u = 0; u < T::DTILES / 2; u++) o[u][0] = o[u][1] = o[u][2] = o[u][3] = 0.f;
             m0 = m1 = -INFINITY;
             l0 = l1 = 0.f;
-            __syncthreads();   // osm becomes the score-exchange buffer
         }
 
         // wait for the slab
@@ -846,14 +866,17 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const DecodePara
                         const int base = T::VCW * c + 4 * uu;
                         const int da = base + 4 * T::VCH * (r >> 1) + (r & 1);   // logical row r
                         const int db = da + 2;                                    // logical row r + 8
+                        // head n's row is stored with d ^ (n << 2), which spreads the
+                        // four heads a warp writes over different banks
                         float* oa0 = osm + (2 * j) * D;
                         float* oa1 = osm + (2 * j + 1) * D;
+                        const int x0 = (2 * j) << 2, x1 = (2 * j + 1) << 2;
                         if (w == 0) {
-                            oa0[da] = o[ul][0] * f0; oa1[da] = o[ul][1] * f1;
-                            oa0[db] = o[ul][2] * f0; oa1[db] = o[ul][3] * f1;
+                            oa0[da ^ x0] = o[ul][0] * f0; oa1[da ^ x1] = o[ul][1] * f1;
+                            oa0[db ^ x0] = o[ul][2] * f0; oa1[db ^ x1] = o[ul][3] * f1;
                         } else {
-                            oa0[da] += o[ul][0] * f0; oa1[da] += o[ul][1] * f1;
-                            oa0[db] += o[ul][2] * f0; oa1[db] += o[ul][3] * f1;
+                            oa0[da ^ x0] += o[ul][0] * f0; oa1[da ^ x1] += o[ul][1] * f1;
+                            oa0[db ^ x0] += o[ul][2] * f0; oa1[db ^ x1] += o[ul][3] * f1;
                         }
                     }
                 }
@@ -876,7 +899,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const DecodePara
                     const float inv = whole ? ((Ls > 0.f) ? p.o_mult / Ls : 0.f) : 1.f;
                     float x[8];
 #pragma unroll
-                    for (int e = 0; e < T::EPL; e++) x[e] = osm[nh * D + lane * T::EPL + e] * inv;
+                    for (int e = 0; e < T::EPL; e++) x[e] = osm[nh * D + ((lane * T::EPL + e) ^ (nh << 2))] * inv;
                     if constexpr (D == 256) {
                         if (p.rot_v) fwht256_warp(x, lane);
                     }
@@ -964,9 +987,10 @@ bool decode_supported(int fmt, int D) {
     return D == 128 || D == 256;
 }
 
-static size_t fixed_smem(int D, int B, int pid_cap) {
+static size_t fixed_smem(int D, int B, int pid_cap, int qs) {
     const size_t osm = 8 * (size_t)D * 4 > 8192 ? 8 * (size_t)D * 4 : 8192;
-    return 8 * kMaxStages + 4 * kMaxStages + 32 + osm + 4 * 16 * 4 + 16 * 4 + 16 + 4 * (size_t)(B + 1) +
+    const size_t qst = 8 * (size_t)D * 2 * qs;
+    return 8 * kMaxStages + 4 * kMaxStages + 32 + osm + qst + 4 * 16 * 4 + 16 * 4 + 16 + 4 * (size_t)(B + 1) +
            4 * (size_t)pid_cap + 128;
 }
 
@@ -982,17 +1006,22 @@ cudaError_t plan_decode(const Layout& L, int B, int HB, int max_seq_len, DecodeP
     if (!kern) return cudaErrorInvalidValue;
     const int64_t pages = (max_seq_len + L.P - 1) / L.P;
     const int64_t work = (int64_t)B * pages * L.H * HB > 0 ? (int64_t)B * pages * L.H * HB : 1;
-    // two CTAs per SM when three stages fit, else one CTA with a deeper pipeline
+    // two CTAs per SM when three stages fit, else one CTA with a deeper pipeline;
+    // the shared memory left over holds the preloaded page ids
+    constexpr int kMinPids = 64;
     for (int ctas = 2; ctas >= 1; ctas--) {
         const int64_t grid = (int64_t)sms * ctas < work ? (int64_t)sms * ctas : work;
-        int64_t cap = (work + grid - 1) / grid + 1;
-        if (cap > 4096) cap = 4096;
-        const size_t fixed = fixed_smem(L.D, B, (int)cap);
+        const size_t fixed = fixed_smem(L.D, B, kMinPids, L.kk == RK_BF16RAW ? 2 : 1);
         const int64_t budget = ctas == 2 ? (int64_t)smem_sm / 2 - 1024 : (int64_t)smem_blk;
         int64_t stages = (budget - (int64_t)fixed) / L.slab;
         if (stages > 6) stages = 6;
         if (stages < (ctas == 2 ? 3 : 2)) continue;
-        const size_t smem = (((size_t)stages * L.slab + 127) & ~(size_t)127) + fixed;
+        const int64_t stage_bytes = ((int64_t)stages * L.slab + 127) & ~(int64_t)127;
+        int64_t cap = (work + grid - 1) / grid + 1;                  // pages of the largest range
+        const int64_t room = kMinPids + (budget - (int64_t)fixed - stage_bytes) / 4;
+        if (cap > room) cap = room;
+        if (cap > 4096) cap = 4096;
+        const size_t smem = (size_t)stage_bytes + fixed + 4 * (size_t)(cap - kMinPids);
         if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
             return e;
         int resident = 0;
