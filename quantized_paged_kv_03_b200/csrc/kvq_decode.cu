@@ -378,8 +378,21 @@ struct Producer {
     int issued;
 };
 
+// CTAs per SM a decode kernel is compiled for.  Three (24 warps, registers
+// capped at 85 per thread) where a 64-token page slab is small enough for three
+// CTAs to keep three stages each in shared memory and the head_dim-128 state
+// fits the cap; two otherwise (head_dim 256 needs the registers, MXFP8 has
+// 128-token slabs, BF16 slabs are 32 KB).
+__host__ __device__ constexpr int decode_ctas(int kk, int vk, int D) {
+    return (D == 128 && kk != RK_E4M3_MX32 &&
+            64 * (row_code_bytes(kk, D) + row_scale_bytes(kk, D) + row_code_bytes(vk, D) + row_scale_bytes(vk, D)) <=
+                20 * 1024)
+               ? 3
+               : 2;
+}
+
 template <int KK, int KV, int D>
-__global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_kernel(const DecodeParams p) {
     using T = DecTraits<KK, KV, D>;
     extern __shared__ __align__(128) uint8_t smem[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -1009,13 +1022,13 @@ cudaError_t plan_decode(const Layout& L, int B, int HB, int max_seq_len, DecodeP
     // two CTAs per SM when three stages fit, else one CTA with a deeper pipeline;
     // the shared memory left over holds the preloaded page ids
     constexpr int kMinPids = 64;
-    for (int ctas = 2; ctas >= 1; ctas--) {
+    for (int ctas = decode_ctas(L.kk, L.vk, L.D); ctas >= 1; ctas--) {
         const int64_t grid = (int64_t)sms * ctas < work ? (int64_t)sms * ctas : work;
         const size_t fixed = fixed_smem(L.D, B, kMinPids, L.kk == RK_BF16RAW ? 2 : 1);
-        const int64_t budget = ctas == 2 ? (int64_t)smem_sm / 2 - 1024 : (int64_t)smem_blk;
+        const int64_t budget = ctas >= 2 ? (int64_t)smem_sm / ctas - 1024 : (int64_t)smem_blk;
         int64_t stages = (budget - (int64_t)fixed) / L.slab;
         if (stages > 6) stages = 6;
-        if (stages < (ctas == 2 ? 3 : 2)) continue;
+        if (stages < (ctas >= 2 ? 3 : 2)) continue;
         const int64_t stage_bytes = ((int64_t)stages * L.slab + 127) & ~(int64_t)127;
         int64_t cap = (work + grid - 1) / grid + 1;                  // pages of the largest range
         const int64_t room = kMinPids + (budget - (int64_t)fixed - stage_bytes) / 4;

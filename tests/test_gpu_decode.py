@@ -34,14 +34,17 @@ CASES = [
     ("bf16", 4, 128, 64, [300, 2], 2, 16),
     ("bf16", 0, 256, 64, [200], 1, 3),
     ("int8_g64", 1, 256, 64, [5000], 1, 24),     # G = 24: three 8-head blocks
+    ("nvfp4_g16", 2, 128, 64, [700, 65, 3], 2, 6),   # 4-bit code words span two q lanes
+    ("int8_g64", 1, 128, 64, [400, 64], 2, 4),
 ]
 
 
 def run_case(fmt, cfg, D, P, lengths, H, Hq, out_fp32=True, seed=11):
     w = workload(cfg, D, P, lengths, H, Hq, seed)
     scales = tensor_scales(w) if fmt == "fp8_tensor" else (1.0, 1.0)
-    c = gpu_cache(w, fmt, 0, scales if fmt == "fp8_tensor" else None)
-    oc = oracle_cache(w, fmt, 0, scales)
+    flags = K.FLAG_NO_ROTATE if D != 256 else 0   # the Hadamard is 256-point
+    c = gpu_cache(w, fmt, flags, scales if fmt == "fp8_tensor" else None)
+    oc = oracle_cache(w, fmt, flags, scales)
     append_all(c, oc, w)
     got = gpu_decode(c, w, out_fp32=out_fp32)
     want = oc.decode(w.q, w.block_table, w.seq_lens, threads=8)
