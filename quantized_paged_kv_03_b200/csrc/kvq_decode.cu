@@ -203,12 +203,12 @@ struct DecTraits {
 
 // Cursor over this CTA's page-heads: (sequence b, head pair hh = h*HB + hb, page).
 struct Cursor {
-    int b, hh, h, hb, page, npages;   // hh = h * HB + hb
+    int b, hh, h, hb, span, nspans;   // hh = h * HB + hb; span = 64-token unit (or page)
 };
 
 __device__ __forceinline__ void cursor_next(Cursor& c, const int* pref, int B, int HH, int HB) {
-    if (++c.page < c.npages) return;
-    c.page = 0;
+    if (++c.span < c.nspans) return;
+    c.span = 0;
     if (++c.hh < HH) {
         if (++c.hb == HB) {
             c.hb = 0;
@@ -220,7 +220,7 @@ __device__ __forceinline__ void cursor_next(Cursor& c, const int* pref, int B, i
     do {
         c.b++;
     } while (c.b < B && pref[c.b + 1] == pref[c.b]);
-    c.npages = (c.b < B) ? pref[c.b + 1] - pref[c.b] : 0;
+    c.nspans = (c.b < B) ? pref[c.b + 1] - pref[c.b] : 0;
 }
 
 __device__ __forceinline__ void cursor_locate(Cursor& c, int64_t w, const int* pref, int B, int HH, int HB) {
@@ -232,18 +232,48 @@ __device__ __forceinline__ void cursor_locate(Cursor& c, int64_t w, const int* p
     }
     while (lo < B - 1 && pref[lo + 1] == pref[lo]) lo++;   // skip empty sequences
     c.b = lo;
-    c.npages = pref[lo + 1] - pref[lo];
+    c.nspans = pref[lo + 1] - pref[lo];
     int64_t idx = w - (int64_t)pref[lo] * HH;
-    c.hh = (int)(idx / c.npages);
-    c.page = (int)(idx % c.npages);
+    c.hh = (int)(idx / c.nspans);
+    c.span = (int)(idx % c.nspans);
     c.h = c.hh / HB;
     c.hb = c.hh % HB;
 }
 
-// CTA owning page-head w when W page-heads are cut into G equal ranges.
-__device__ __forceinline__ int owner_of(int64_t w, int64_t W, int G) {
-    return (int)(((w + 1) * G + W - 1) / W) - 1;
-}
+// How the units are cut between the G CTAs: into ranges of equal cost, where
+// a unit costs 1 and every segment (sequence, kv-head, head block) adds `c` at
+// its start -- the fixed work of starting and finishing a segment, so that CTAs
+// whose range touches many short segments get fewer units.  Cost positions:
+// sequence b starts at pref[b] * HH + c * HH * b (empty sequences keep their
+// segment costs; they only shift positions), segment hh of b occupies
+// c + n_b positions, its unit u sits at position c + u of them.
+struct Partition {
+    const int* pref;
+    int B, HH, c, G;
+    int64_t W, C;   // units, total cost
+
+    __device__ int64_t seq_cost(int b) const { return (int64_t)pref[b] * HH + (int64_t)c * HH * b; }
+    // first unit at or after cost position X
+    __device__ int64_t unit_at(int64_t X) const {
+        if (X >= C) return W;
+        int lo = 0, hi = B - 1;   // largest b with seq_cost(b) <= X
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (seq_cost(mid) <= X) lo = mid;
+            else hi = mid - 1;
+        }
+        const int nb = pref[lo + 1] - pref[lo];
+        const int64_t local = X - seq_cost(lo), len = (int64_t)nb + c;
+        const int64_t hh = local / len, r = local - hh * len;
+        return (int64_t)pref[lo] * HH + hh * nb + (r > c ? r - c : 0);
+    }
+    __device__ int64_t start(int i) const { return unit_at((int64_t)i * C / G); }
+    // CTA whose range holds unit w = (b, hh, u)
+    __device__ int owner(int b, int hh, int u) const {
+        const int64_t x = seq_cost(b) + (int64_t)hh * (pref[b + 1] - pref[b] + c) + c + u;
+        return (int)(((x + 1) * G + C - 1) / C) - 1;
+    }
+};
 
 // Store EPL consecutive output values (fp32 or bf16) at element offset `ob`.
 template <int EPL>
@@ -299,7 +329,7 @@ __device__ __forceinline__ bool grid_barrier(unsigned* bar, unsigned G, int* fla
 // produces float4 outputs [o0, o1) of the segment's gv x D/4.
 template <int D>
 __device__ __forceinline__ void merge_segment(const DecodeParams& p, int b, int h, int hb, int64_t seg_w0,
-                                              int i_first, int i_last, int64_t W, int G, float* fin) {
+                                              int i_first, int i_last, const Partition& part, float* fin) {
     const int tid = threadIdx.x;
     const int P = i_last - i_first + 1;
     const int j = (int)blockIdx.x - i_first;
@@ -308,7 +338,7 @@ __device__ __forceinline__ void merge_segment(const DecodeParams& p, int b, int 
     const int o0 = (int)((int64_t)j * NU / P), o1 = (int)((int64_t)(j + 1) * NU / P);
     auto part_of = [&](int k) -> const float* {
         const int i = i_first + k;
-        const int64_t start = (int64_t)i * W / G;
+        const int64_t start = part.start(i);
         return p.partials + ((int64_t)i * 2 + (start >= seg_w0 ? 0 : 1)) * (16 + 8 * D);
     };
     // segment max and sum per head: 16 lanes per head (threads 0..127)
@@ -379,10 +409,11 @@ struct Producer {
 };
 
 // CTAs per SM a decode kernel is compiled for.  Three (24 warps, registers
-// capped at 85 per thread) where a 64-token page slab is small enough for three
-// CTAs to keep three stages each in shared memory and the head_dim-128 state
-// fits the cap; two otherwise (head_dim 256 needs the registers, MXFP8 has
-// 128-token slabs, BF16 slabs are 32 KB).
+// capped at 80 per thread) where a 64-token page is small enough for three CTAs
+// to keep three stages each in shared memory and the head_dim-128 state fits
+// the cap; two otherwise (head_dim 256 needs the registers, BF16 pages are
+// 32 KB, and MXFP8's 128-token pages run faster whole at two CTAs than split
+// into 64-token units at three).
 __host__ __device__ constexpr int decode_ctas(int kk, int vk, int D) {
     return (D == 128 && kk != RK_E4M3_MX32 &&
             64 * (row_code_bytes(kk, D) + row_scale_bytes(kk, D) + row_code_bytes(vk, D) + row_scale_bytes(vk, D)) <=
@@ -399,11 +430,12 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
     const int r = lane >> 2, j = lane & 3;
     const int tw = warp & 3, hf = warp >> 2;     // tile slot, head_dim half
     const int H = p.L.H, P = p.L.P, HB = p.HB, HH = H * HB, B = p.B;
-    const int64_t slab = p.L.slab;
+    const int64_t slab = p.L.slab;            // page slab stride in HBM
+    const SpanLayout& U = p.U;                // what one stage holds
     const int NS = p.stages;
 
     // shared memory carve-up
-    size_t off = ((size_t)NS * slab + 127) & ~(size_t)127;
+    size_t off = ((size_t)NS * U.bytes + 127) & ~(size_t)127;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + off);   // full[stage]
     off += 8 * kMaxStages;
     int* rel = reinterpret_cast<int*>(smem + off);               // release count[stage]
@@ -425,20 +457,22 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
     off += 4 * (size_t)(B + 1);
     int* pids = reinterpret_cast<int*>(smem + off);      // [pid_cap] page ids of this CTA's range
     volatile int* abort_flag = flags;
+    // units of a sequence of L tokens (at most max_pages pages of it)
+    auto n_units = [&](int L) {
+        const int u = L > 0 ? (L + U.sp - 1) / U.sp : 0;
+        return min(u, p.max_pages << U.lg_up);
+    };
 
-    // ---- page prefix over the batch (block scan)
+    // ---- unit prefix over the batch (block scan): units of sequence b are
+    // pref[b] .. pref[b + 1] - 1
     {
         const int per = (B + kDecThreads - 1) / kDecThreads;
         const int b0 = tid * per, b1 = min(B, b0 + per);
         int local = 0;
         for (int b = b0; b < b1; b++) {
-            int L = p.seq_lens[b];
-            int np = L > 0 ? (L + P - 1) / P : 0;
-            if (np > p.max_pages) {
-                np = p.max_pages;
-                atomicOr(p.status, kStatusBadPage);
-            }
-            local += np;
+            const int L = p.seq_lens[b];
+            if (L > 0 && (L + P - 1) / P > p.max_pages) atomicOr(p.status, kStatusBadPage);
+            local += n_units(L);
         }
         int incl = local;
 #pragma unroll
@@ -454,9 +488,7 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
         int run = base + incl - local;
         for (int b = b0; b < b1; b++) {
             pref[b] = run;
-            int L = p.seq_lens[b];
-            int np = L > 0 ? (L + P - 1) / P : 0;
-            run += min(np, p.max_pages);
+            run += n_units(p.seq_lens[b]);
         }
         if (tid == kDecThreads - 1) pref[B] = run;
         if (B == 0 && tid == 0) pref[0] = 0;
@@ -478,37 +510,60 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
     if (W == 0) return;
     const int G = (int)(((int64_t)gridDim.x < W) ? (int64_t)gridDim.x : W);
     if ((int)blockIdx.x >= G) return;
-    const int64_t w0 = (int64_t)blockIdx.x * W / G, w1 = (int64_t)(blockIdx.x + 1) * W / G;
+    Partition part;
+    part.pref = pref;
+    part.B = B;
+    part.HH = HH;
+    part.c = p.seg_cost;
+    part.G = G;
+    part.W = W;
+    part.C = part.seq_cost(B);
+    const int64_t w0 = part.start(blockIdx.x), w1 = part.start(blockIdx.x + 1);
     const int n = (int)(w1 - w0);
 
     // ---- page ids of this CTA's range, loaded in parallel up front so that a
     // refill never waits on a block-table read
-    auto page_id = [&](int64_t w) {
-        Cursor c;
-        cursor_locate(c, w, pref, B, HH, HB);
-        int pid = p.block_table[(int64_t)c.b * p.max_pages + c.page];
+    auto checked = [&](int pid) {
         if (pid < 0 || pid >= p.L.num_pages) {
             atomicOr(p.status, kStatusBadPage);
             pid = 0;
         }
         return pid;
     };
-    for (int k = tid; k < n && k < p.pid_cap; k += kDecThreads) pids[k] = page_id(w0 + k);
-    __syncthreads();
+    auto pid_at = [&](const Cursor& c) {
+        return checked(p.block_table[(int64_t)c.b * p.max_pages + (c.span >> U.lg_up)]);
+    };
+    auto page_id = [&](int64_t w) {
+        Cursor c;
+        cursor_locate(c, w, pref, B, HH, HB);
+        return pid_at(c);
+    };
 
-    // ---- producer: the slab of the next page-head into a free stage
-    auto issue = [&](int s) {
+    // ---- producer: the next unit into a free stage (one copy of a whole page
+    // slab, or the unit's rows of each of the slab's four arrays)
+    auto issue = [&](int s, int pid) {
         Cursor& pc = prod->c;
-        const int k = prod->issued;
-        const int pid = (k < p.pid_cap) ? pids[k] : page_id(w0 + k);
         const uint8_t* src = p.slabs + ((int64_t)pid * H + pc.h) * slab;
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        uint32_t bar = smem_u32(&bars[s]);
-        mbar_expect_tx(bar, (uint32_t)slab);
-        bulk_g2s(smem_u32(smem + (size_t)s * slab), src, (uint32_t)slab, bar);
+        const uint32_t bar = smem_u32(&bars[s]);
+        const uint32_t dst = smem_u32(smem + (size_t)s * U.bytes);
+        if (U.lg_up == 0) {
+            mbar_expect_tx(bar, (uint32_t)slab);
+            bulk_g2s(dst, src, (uint32_t)slab, bar);
+        } else {
+            const int64_t r0 = (int64_t)(pc.span & ((1 << U.lg_up) - 1)) * U.sp;
+            const uint32_t nk = U.sp * p.L.kc, nks = U.sp * p.L.ks, nv = U.sp * p.L.vc, nvs = U.sp * p.L.vs;
+            mbar_expect_tx(bar, nk + nks + nv + nvs);
+            bulk_g2s(dst, src + r0 * p.L.kc, nk, bar);
+            if (nks) bulk_g2s(dst + (uint32_t)U.off_ks, src + p.L.off_ks + r0 * p.L.ks, nks, bar);
+            bulk_g2s(dst + (uint32_t)U.off_vc, src + p.L.off_vc + r0 * p.L.vc, nv, bar);
+            if (nvs) bulk_g2s(dst + (uint32_t)U.off_vs, src + p.L.off_vs + r0 * p.L.vs, nvs, bar);
+        }
         cursor_next(pc, pref, B, HH, HB);
         prod->issued++;
     };
+    // thread 0 starts the ring with its own block-table reads (all in flight at
+    // once) while the other threads preload the range's page ids
     if (tid == 0) {
         for (int s = 0; s < NS; s++) {
             mbar_init(smem_u32(&bars[s]), 1);
@@ -517,14 +572,27 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         cursor_locate(prod->c, w0, pref, B, HH, HB);
         prod->issued = 0;
-        for (int s = 0; s < NS && s < n; s++) issue(s);
+        int first[kMaxStages];
+        Cursor c = prod->c;
+#pragma unroll
+        for (int s = 0; s < kMaxStages; s++) {
+            first[s] = 0;
+            if (s < NS && s < n) {
+                first[s] = p.block_table[(int64_t)c.b * p.max_pages + (c.span >> U.lg_up)];
+                cursor_next(c, pref, B, HH, HB);
+            }
+        }
+#pragma unroll
+        for (int s = 0; s < kMaxStages; s++)
+            if (s < NS && s < n) issue(s, checked(first[s]));
     }
+    for (int k = tid; k < n && k < p.pid_cap; k += kDecThreads) pids[k] = page_id(w0 + k);
     __syncthreads();
 
     // ---- consumer state (warp pair: tile slot tw, head_dim half hf)
     Cursor cc;
     cursor_locate(cc, w0, pref, B, HH, HB);
-    const int tiles = P >> 4;    // 16-token tiles per page
+    const int tiles = U.sp >> 4;    // 16-token tiles per unit
     int s = 0;                   // stage of page i
     uint32_t ph = 0;             // mbarrier phase of that stage's current use
     int seq_len = 0;
@@ -557,13 +625,13 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
         else if constexpr (KV == RK_E4M3_MX32) vsoff[cl] = r * T::VS + c;
         else vsoff[cl] = r * T::VS;
     }
-    const uint32_t off_ks = (uint32_t)p.L.off_ks, off_vc = (uint32_t)p.L.off_vc, off_vs = (uint32_t)p.L.off_vs;
+    const uint32_t off_ks = (uint32_t)U.off_ks, off_vc = (uint32_t)U.off_vc, off_vs = (uint32_t)U.off_vs;
     float4* xmine = xbuf + (tw * 2 + hf) * 32 + lane;          // parity 0; parity 1 is +8*32
     const float4* xother = xbuf + (tw * 2 + (hf ^ 1)) * 32 + lane;
 
     for (int i = 0; i < n; i++) {
         const int b = cc.b, h = cc.h, hb = cc.hb;
-        if (i == 0 || cc.page == 0) {
+        if (i == 0 || cc.span == 0) {
             // ---- segment start: q rows of this 8-head block, rotated and scaled
             seg_first = (i == 0);
             seq_len = p.seq_lens[b];
@@ -636,13 +704,16 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
         (void)mbar_wait(smem_u32(&bars[s]), ph, abort_flag);
 
         // ---- this pair's 16-token tiles of the page
-        const uint32_t stg = (uint32_t)s * (uint32_t)slab;   // byte offset of the stage
+        const uint32_t stg = (uint32_t)s * (uint32_t)U.bytes;   // byte offset of the stage
 
-        if (p.k_new != nullptr && cc.page == cc.npages - 1) {
+        if (p.k_new != nullptr && cc.span == cc.nspans - 1) {
             // fused append: the sequence's newest token (position seq_len - 1) lies
-            // in its last page.  Quantise it into this stage, over whatever the copy
-            // brought, and into the cache (one head block writes the cache).
-            const int t = (seq_len - 1) - cc.page * P;
+            // in its last unit.  Quantise it into this stage (row t of the unit),
+            // over whatever the copy brought, and into the cache (row tp of the
+            // page; one head block writes the cache).  t and tp differ by a
+            // multiple of 64, so the row's chunk permutation is the same.
+            const int t = (seq_len - 1) - cc.span * U.sp;
+            const int tp = t + (cc.span & ((1 << U.lg_up) - 1)) * U.sp;
             if (warp < 2) {
                 const int pid = (i < p.pid_cap) ? pids[i] : page_id(w0 + i);
                 uint8_t* g = p.slabs + ((int64_t)pid * H + h) * slab;
@@ -651,20 +722,21 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
                     const uint16_t* src = p.k_new + ((int64_t)b * H + h) * D;
                     quantize_row<KK, D>(src, p.rot_k, p.k_scale, st + t * T::KC, st + off_ks + t * T::KS, t, lane);
                     if (hb == 0)
-                        quantize_row<KK, D>(src, p.rot_k, p.k_scale, g + t * T::KC, g + off_ks + t * T::KS, t, lane);
+                        quantize_row<KK, D>(src, p.rot_k, p.k_scale, g + tp * T::KC, g + p.L.off_ks + tp * T::KS, tp,
+                                            lane);
                 } else {
                     const uint16_t* src = p.v_new + ((int64_t)b * H + h) * D;
                     quantize_row<KV, D>(src, p.rot_v, p.v_scale, st + off_vc + t * T::VC, st + off_vs + t * T::VS,
                                         t, lane);
                     if (hb == 0)
-                        quantize_row<KV, D>(src, p.rot_v, p.v_scale, g + off_vc + t * T::VC, g + off_vs + t * T::VS,
-                                            t, lane);
+                        quantize_row<KV, D>(src, p.rot_v, p.v_scale, g + p.L.off_vc + tp * T::VC,
+                                            g + p.L.off_vs + tp * T::VS, tp, lane);
                 }
             }
             asm volatile("bar.sync 5, %0;" ::"r"(kDecThreads) : "memory");
         }
         for (int mt = tw; mt < tiles; mt += 4) {
-            const int valid = seq_len - (cc.page * P + mt * 16);
+            const int valid = seq_len - (cc.span * U.sp + mt * 16);
             if (valid <= 0) break;   // same decision in both warps of the pair
             const uint32_t kt = stg + mt * 16 * T::KC, kst = stg + off_ks + mt * 16 * T::KS;
             const uint32_t vt = stg + off_vc + mt * 16 * T::VC, vst = stg + off_vs + mt * 16 * T::VS;
@@ -831,11 +903,12 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
             if (old == kDecThreads / 32 - 1) {
                 rel[s] = 0;
                 __threadfence_block();
-                if (prod->issued < n && !*abort_flag) issue(s);
+                const int k = prod->issued;
+                if (k < n && !*abort_flag) issue(s, (k < p.pid_cap) ? pids[k] : page_id(w0 + k));
             }
         }
 
-        const bool seg_end = (i == n - 1) || (cc.page == cc.npages - 1);
+        const bool seg_end = (i == n - 1) || (cc.span == cc.nspans - 1);
         if (seg_end) {
             // ---- merge the warps: max, rescaled sums, rescaled outputs.  The two
             // warps of a pair hold the same (m, l); the half-0 warp reports them.
@@ -900,8 +973,8 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
             // a range boundary leaves its unnormalised output as this CTA's partial
             // (rotated back already: the Hadamard is linear, so merging commutes
             // with it) for the merge after the grid barrier.
-            const int64_t seg_w0 = (int64_t)pref[b] * HH + (int64_t)cc.hh * cc.npages;
-            const bool whole = (seg_w0 >= w0) && (seg_w0 + cc.npages <= w1);
+            const int64_t seg_w0 = (int64_t)pref[b] * HH + (int64_t)cc.hh * cc.nspans;
+            const bool whole = (seg_w0 >= w0) && (seg_w0 + cc.nspans <= w1);
             float* part = p.partials + ((int64_t)blockIdx.x * 2 + (seg_first ? 0 : 1)) * (16 + 8 * D);
             if (!whole && tid < 16) part[tid] = fin[tid];
             {
@@ -958,14 +1031,14 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
         Cursor c0, c1;
         cursor_locate(c0, w0, pref, B, HH, HB);
         cursor_locate(c1, w1 - 1, pref, B, HH, HB);
-        for (int k = 0; k < 2; k++) {
+        for (int k = 0; k < (n > 0 ? 2 : 0); k++) {
             const Cursor& c = k == 0 ? c0 : c1;
             if (k == 1 && c1.b == c0.b && c1.hh == c0.hh) break;
-            const int64_t seg_w0 = (int64_t)pref[c.b] * HH + (int64_t)c.hh * c.npages;
-            if (seg_w0 >= w0 && seg_w0 + c.npages <= w1) continue;     // whole: already stored
-            const int i_first = owner_of(seg_w0, W, G);
-            const int i_last = owner_of(seg_w0 + c.npages - 1, W, G);
-            merge_segment<D>(p, c.b, c.h, c.hb, seg_w0, i_first, i_last, W, G, fin);
+            const int64_t seg_w0 = (int64_t)pref[c.b] * HH + (int64_t)c.hh * c.nspans;
+            if (seg_w0 >= w0 && seg_w0 + c.nspans <= w1) continue;     // whole: already stored
+            const int i_first = part.owner(c.b, c.hh, 0);
+            const int i_last = part.owner(c.b, c.hh, c.nspans - 1);
+            merge_segment<D>(p, c.b, c.h, c.hb, seg_w0, i_first, i_last, part, fin);
         }
     }
 }
@@ -1017,36 +1090,43 @@ cudaError_t plan_decode(const Layout& L, int B, int HB, int max_seq_len, DecodeP
     if ((e = cudaDeviceGetAttribute(&smem_blk, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess) return e;
     const void* kern = decode_kernel_for(L.fmt, L.D);
     if (!kern) return cudaErrorInvalidValue;
-    const int64_t pages = (max_seq_len + L.P - 1) / L.P;
-    const int64_t work = (int64_t)B * pages * L.H * HB > 0 ? (int64_t)B * pages * L.H * HB : 1;
-    // two CTAs per SM when three stages fit, else one CTA with a deeper pipeline;
-    // the shared memory left over holds the preloaded page ids
+    // The most CTAs per SM the kernel allows, each with at least three stages
+    // (one CTA: two).  A stage holds a whole page if that fits, else (128- and
+    // 256-token pages) a 64-token unit.  The shared memory left over holds the
+    // preloaded page ids.
     constexpr int kMinPids = 64;
+    const int lg_unit = L.P == 128 ? 1 : L.P == 256 ? 2 : 0;
     for (int ctas = decode_ctas(L.kk, L.vk, L.D); ctas >= 1; ctas--) {
-        const int64_t grid = (int64_t)sms * ctas < work ? (int64_t)sms * ctas : work;
         const size_t fixed = fixed_smem(L.D, B, kMinPids, L.kk == RK_BF16RAW ? 2 : 1);
         const int64_t budget = ctas >= 2 ? (int64_t)smem_sm / ctas - 1024 : (int64_t)smem_blk;
-        int64_t stages = (budget - (int64_t)fixed) / L.slab;
-        if (stages > 6) stages = 6;
-        if (stages < (ctas >= 2 ? 3 : 2)) continue;
-        const int64_t stage_bytes = ((int64_t)stages * L.slab + 127) & ~(int64_t)127;
-        int64_t cap = (work + grid - 1) / grid + 1;                  // pages of the largest range
-        const int64_t room = kMinPids + (budget - (int64_t)fixed - stage_bytes) / 4;
-        if (cap > room) cap = room;
-        if (cap > 4096) cap = 4096;
-        const size_t smem = (size_t)stage_bytes + fixed + 4 * (size_t)(cap - kMinPids);
-        if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
-            return e;
-        int resident = 0;
-        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident, kern, kDecThreads, smem)) != cudaSuccess)
-            return e;
-        if (resident < ctas) continue;
-        plan->stages = (int)stages;
-        plan->threads = kDecThreads;
-        plan->pid_cap = (int)cap;
-        plan->smem = smem;
-        plan->grid = (int)grid;
-        return cudaSuccess;
+        for (int lg_up = 0; lg_up <= lg_unit; lg_up += (lg_unit ? lg_unit : 1)) {
+            const SpanLayout U = make_span(L, lg_up);
+            const int64_t units = (max_seq_len + U.sp - 1) / U.sp;
+            const int64_t work = (int64_t)B * units * L.H * HB > 0 ? (int64_t)B * units * L.H * HB : 1;
+            const int64_t grid = (int64_t)sms * ctas < work ? (int64_t)sms * ctas : work;
+            int64_t stages = (budget - (int64_t)fixed) / U.bytes;
+            if (stages > 6) stages = 6;
+            if (stages < (ctas >= 2 ? 3 : 2)) continue;
+            const int64_t stage_bytes = ((int64_t)stages * U.bytes + 127) & ~(int64_t)127;
+            int64_t cap = (work + grid - 1) / grid + 1;                  // units of the largest range
+            const int64_t room = kMinPids + (budget - (int64_t)fixed - stage_bytes) / 4;
+            if (cap > room) cap = room;
+            if (cap > 4096) cap = 4096;
+            const size_t smem = (size_t)stage_bytes + fixed + 4 * (size_t)(cap - kMinPids);
+            if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+                return e;
+            int resident = 0;
+            if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident, kern, kDecThreads, smem)) != cudaSuccess)
+                return e;
+            if (resident < ctas) continue;
+            plan->stages = (int)stages;
+            plan->threads = kDecThreads;
+            plan->pid_cap = (int)cap;
+            plan->smem = smem;
+            plan->grid = (int)grid;
+            plan->lg_up = lg_up;
+            return cudaSuccess;
+        }
     }
     return cudaErrorInvalidConfiguration;
 }
@@ -1071,7 +1151,11 @@ void decode_workspace_zero_region(const Layout& L, int B, int HB, int grid, size
 cudaError_t launch_decode(const DecodeParams& p, const DecodePlan& plan, cudaStream_t s) {
     const void* k = decode_kernel_for(p.L.fmt, p.L.D);
     if (!k) return cudaErrorInvalidValue;
-    void* args[] = {const_cast<DecodeParams*>(&p)};
+    DecodeParams q = p;
+    q.U = make_span(p.L, plan.lg_up);
+    // cost of a segment's start and end in units (about four 64-token units)
+    q.seg_cost = q.U.sp >= 256 ? 1 : 256 / q.U.sp;
+    void* args[] = {&q};
     // cooperative: the merge after the grid barrier needs every CTA resident
     return cudaLaunchCooperativeKernel(k, dim3(plan.grid), dim3(plan.threads), args, plan.smem, s);
 }

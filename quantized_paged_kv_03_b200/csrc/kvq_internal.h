@@ -34,8 +34,29 @@ struct DequantParams {
     float *k_out, *v_out;
 };
 
+// The unit a decode stage holds: a whole page (one copy of the page slab), or,
+// for 128- and 256-token pages too large for the stage ring, 64 tokens of it
+// (four copies: those rows of K codes, K scales, V codes, V scales).  A unit's
+// stage layout is the page layout for its row count.
+struct SpanLayout {
+    int lg_up, sp;                       // log2(units per page), tokens per unit
+    int off_ks, off_vc, off_vs, bytes;   // the unit's arrays in its stage
+};
+inline SpanLayout make_span(const Layout& L, int lg_up) {
+    SpanLayout u;
+    u.lg_up = lg_up;
+    u.sp = L.P >> u.lg_up;
+    u.off_ks = (int)align16((int64_t)u.sp * L.kc);
+    u.off_vc = u.off_ks + (int)align16((int64_t)u.sp * L.ks);
+    u.off_vs = u.off_vc + (int)align16((int64_t)u.sp * L.vc);
+    u.bytes = u.off_vs + (int)align16((int64_t)u.sp * L.vs);
+    return u;
+}
+
 struct DecodeParams {
     Layout L;
+    SpanLayout U;                // set by the launch from L
+    int seg_cost;                // set by the launch: a segment's fixed cost in units
     uint8_t* slabs;              // first slab of the layer (written only by the fused append)
     const uint16_t* q;           // bf16 [B][Hq][D]
     int Hq, G, HB;               // query heads, GQA group, 8-head blocks per kv-head
@@ -66,6 +87,7 @@ cudaError_t launch_encode(int code, const float* x, int64_t n, uint8_t* out, cud
 // Decode: grid / smem plan for a layout (host side), then the launch.
 struct DecodePlan {
     int grid, stages, threads, pid_cap;
+    int lg_up;                   // log2(stage units per page)
     size_t smem;
 };
 cudaError_t plan_decode(const Layout& L, int B, int HB, int max_seq_len, DecodePlan* plan);

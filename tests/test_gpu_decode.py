@@ -36,6 +36,11 @@ CASES = [
     ("int8_g64", 1, 256, 64, [5000], 1, 24),     # G = 24: three 8-head blocks
     ("nvfp4_g16", 2, 128, 64, [700, 65, 3], 2, 6),   # 4-bit code words span two q lanes
     ("int8_g64", 1, 128, 64, [400, 64], 2, 4),
+    # pages staged in 64-token units (128 and 256 tokens) and whole small pages
+    ("int8_g64", 1, 256, 128, [300, 129, 64, 1], 2, 8),
+    ("nvfp4_g16", 2, 256, 256, [700, 255, 1], 1, 6),
+    ("fp8_tensor", 4, 128, 32, [100, 33, 1], 2, 8),
+    ("k8v4", 3, 256, 128, [500, 130], 1, 6),
 ]
 
 
@@ -128,7 +133,8 @@ def test_decode_many_sequences_balanced_split():
     ("k8v4", 3, 256, 64, [2000, 129], 2, 12),
     ("mxfp8_g32", 4, 128, 128, [600, 128, 1], 2, 16),
     ("fp8_tensor", 4, 128, 64, [512, 77], 2, 16),
-    ("bf16", 4, 128, 64, [300, 2], 2, 16)])
+    ("bf16", 4, 128, 64, [300, 2], 2, 16),
+    ("int8_g64", 1, 256, 256, [700, 193, 64], 1, 8)])
 def test_fused_append_decode_equals_append_then_decode(fmt, cfg, D, P, lengths, H, Hq):
     """kvq_append_decode stores the same codes as kvq_append and returns the
     same output as kvq_decode_attention run after it."""
