@@ -326,80 +326,62 @@ __device__ __forceinline__ bool grid_barrier(unsigned* bar, unsigned G, int* fla
 
 // Merge share `j` of the partials of one cut segment (CTAs i_first..i_last
 // each left (max, sum, unnormalised output) for up to 8 query heads): this CTA
-// produces float4 outputs [o0, o1) of the segment's gv x D/4.
+// produces float4 outputs [o0, o1) of the segment's gv x D/4.  One pass: each
+// output's threads fold the parts in with a running (max, sum, output) -- the
+// log-sum-exp merge -- then combine their folds by shuffles; no block barrier.
 template <int D>
 __device__ __forceinline__ void merge_segment(const DecodeParams& p, int b, int h, int hb, int64_t seg_w0,
-                                              int i_first, int i_last, const Partition& part, float* fin) {
+                                              int i_first, int i_last, const Partition& part) {
     const int tid = threadIdx.x;
     const int P = i_last - i_first + 1;
     const int j = (int)blockIdx.x - i_first;
     const int gv = min(8, p.G - hb * 8);
     const int NU = gv * (D / 4);
     const int o0 = (int)((int64_t)j * NU / P), o1 = (int)((int64_t)(j + 1) * NU / P);
-    auto part_of = [&](int k) -> const float* {
-        const int i = i_first + k;
-        const int64_t start = part.start(i);
-        return p.partials + ((int64_t)i * 2 + (start >= seg_w0 ? 0 : 1)) * (16 + 8 * D);
-    };
-    // segment max and sum per head: 16 lanes per head (threads 0..127)
-    __syncthreads();
-    if (tid < 128) {
-        const int g = tid >> 4, pl = tid & 15;
-        float M = -INFINITY;
-        for (int k = pl; k < P; k += 16) M = fmaxf(M, __ldcg(part_of(k) + g));
-#pragma unroll
-        for (int m = 1; m < 16; m <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, m));
-        float L = 0.f;
-        for (int k = pl; k < P; k += 16) {
-            const float* pk = part_of(k);
-            const float mk = __ldcg(pk + g);
-            if (mk != -INFINITY) L += exp2f(mk - M) * __ldcg(pk + 8 + g);
-        }
-#pragma unroll
-        for (int m = 1; m < 16; m <<= 1) L += __shfl_xor_sync(0xffffffffu, L, m);
-        if (pl == 0) {
-            fin[g] = M;
-            fin[8 + g] = L;
-        }
-    }
-    __syncthreads();
     const int no = o1 - o0;
-    if (no > 0) {
-        int tpo = 1;
-        while (tpo < 16 && tpo * 2 * no <= kDecThreads) tpo *= 2;
-        const int per_pass = kDecThreads / tpo;
-        for (int ob = o0; ob < o1; ob += per_pass) {
-            const int o = ob + tid / tpo, pl = tid % tpo;
-            const bool valid = o < o1;
-            const int g = valid ? o / (D / 4) : 0, d4 = valid ? o % (D / 4) : 0;
-            const float M = fin[g];
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (valid) {
-                for (int k = pl; k < P; k += tpo) {
-                    const float* pk = part_of(k);
-                    const float mk = __ldcg(pk + g);
-                    const float4 v = __ldcg(reinterpret_cast<const float4*>(pk + 16 + g * D) + d4);
-                    const float wk = (mk == -INFINITY) ? 0.f : exp2f(mk - M);
-                    acc.x = fmaf(wk, v.x, acc.x); acc.y = fmaf(wk, v.y, acc.y);
-                    acc.z = fmaf(wk, v.z, acc.z); acc.w = fmaf(wk, v.w, acc.w);
-                }
-            }
-            for (int m = 1; m < tpo; m <<= 1) {
-                acc.x += __shfl_xor_sync(0xffffffffu, acc.x, m);
-                acc.y += __shfl_xor_sync(0xffffffffu, acc.y, m);
-                acc.z += __shfl_xor_sync(0xffffffffu, acc.z, m);
-                acc.w += __shfl_xor_sync(0xffffffffu, acc.w, m);
-            }
-            if (valid && pl == 0) {
-                const float Ls = fin[8 + g];
-                const float inv = (Ls > 0.f) ? p.o_mult / Ls : 0.f;
-                const float x[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
-                const int64_t oo = ((int64_t)b * p.Hq + h * p.G + hb * 8 + g) * D + 4 * d4;
-                store_out<4>(p, oo, x);
+    if (no <= 0) return;
+    int tpo = 1;   // threads per output, splitting the parts
+    while (tpo < 16 && tpo * 2 * no <= kDecThreads) tpo *= 2;
+    const int per_pass = kDecThreads / tpo;
+    for (int ob = o0; ob < o1; ob += per_pass) {
+        const int o = ob + tid / tpo, pl = tid % tpo;
+        const bool valid = o < o1;
+        const int g = valid ? o / (D / 4) : 0, d4 = valid ? o % (D / 4) : 0;
+        float M = -INFINITY, L = 0.f;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (valid) {
+            for (int k = pl; k < P; k += tpo) {
+                const int i = i_first + k;
+                const float* pk = p.partials + ((int64_t)i * 2 + (part.start(i) >= seg_w0 ? 0 : 1)) * (16 + 8 * D);
+                const float mk = __ldcg(pk + g), lk = __ldcg(pk + 8 + g);
+                const float4 v = __ldcg(reinterpret_cast<const float4*>(pk + 16 + g * D) + d4);
+                if (mk == -INFINITY) continue;
+                const float Mn = fmaxf(M, mk);
+                const float a = (M == -INFINITY) ? 0.f : exp2f(M - Mn), w = exp2f(mk - Mn);
+                acc.x = fmaf(w, v.x, acc.x * a); acc.y = fmaf(w, v.y, acc.y * a);
+                acc.z = fmaf(w, v.z, acc.z * a); acc.w = fmaf(w, v.w, acc.w * a);
+                L = fmaf(w, lk, L * a);
+                M = Mn;
             }
         }
+        for (int m = 1; m < tpo; m <<= 1) {
+            const float M2 = __shfl_xor_sync(0xffffffffu, M, m), L2 = __shfl_xor_sync(0xffffffffu, L, m);
+            const float x2 = __shfl_xor_sync(0xffffffffu, acc.x, m), y2 = __shfl_xor_sync(0xffffffffu, acc.y, m);
+            const float z2 = __shfl_xor_sync(0xffffffffu, acc.z, m), w2 = __shfl_xor_sync(0xffffffffu, acc.w, m);
+            const float Mn = fmaxf(M, M2);
+            const float a = (M == -INFINITY) ? 0.f : exp2f(M - Mn), c = (M2 == -INFINITY) ? 0.f : exp2f(M2 - Mn);
+            acc.x = acc.x * a + x2 * c; acc.y = acc.y * a + y2 * c;
+            acc.z = acc.z * a + z2 * c; acc.w = acc.w * a + w2 * c;
+            L = L * a + L2 * c;
+            M = Mn;
+        }
+        if (valid && pl == 0) {
+            const float inv = (L > 0.f) ? p.o_mult / L : 0.f;
+            const float x[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
+            const int64_t oo = ((int64_t)b * p.Hq + h * p.G + hb * 8 + g) * D + 4 * d4;
+            store_out<4>(p, oo, x);
+        }
     }
-    __syncthreads();
 }
 
 // Shared state of the stage producer (only the warp that issues a copy touches it).
@@ -572,21 +554,17 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         cursor_locate(prod->c, w0, pref, B, HH, HB);
         prod->issued = 0;
-        int first[kMaxStages];
         Cursor c = prod->c;
 #pragma unroll
         for (int s = 0; s < kMaxStages; s++) {
-            first[s] = 0;
             if (s < NS && s < n) {
-                first[s] = p.block_table[(int64_t)c.b * p.max_pages + (c.span >> U.lg_up)];
+                pids[s] = checked(p.block_table[(int64_t)c.b * p.max_pages + (c.span >> U.lg_up)]);
                 cursor_next(c, pref, B, HH, HB);
             }
         }
-#pragma unroll
-        for (int s = 0; s < kMaxStages; s++)
-            if (s < NS && s < n) issue(s, checked(first[s]));
+        for (int s = 0; s < NS && s < n; s++) issue(s, pids[s]);
     }
-    for (int k = tid; k < n && k < p.pid_cap; k += kDecThreads) pids[k] = page_id(w0 + k);
+    for (int k = NS + tid; k < n && k < p.pid_cap; k += kDecThreads) pids[k] = page_id(w0 + k);
     __syncthreads();
 
     // ---- consumer state (warp pair: tile slot tw, head_dim half hf)
@@ -718,19 +696,17 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
                 const int pid = (i < p.pid_cap) ? pids[i] : page_id(w0 + i);
                 uint8_t* g = p.slabs + ((int64_t)pid * H + h) * slab;
                 uint8_t* st = smem + stg;
+                const bool to_cache = (hb == 0);
                 if (warp == 0) {
                     const uint16_t* src = p.k_new + ((int64_t)b * H + h) * D;
-                    quantize_row<KK, D>(src, p.rot_k, p.k_scale, st + t * T::KC, st + off_ks + t * T::KS, t, lane);
-                    if (hb == 0)
-                        quantize_row<KK, D>(src, p.rot_k, p.k_scale, g + tp * T::KC, g + p.L.off_ks + tp * T::KS, tp,
-                                            lane);
+                    quantize_row<KK, D>(src, p.rot_k, p.k_scale, st + t * T::KC, st + off_ks + t * T::KS, t, lane,
+                                        to_cache ? g + tp * T::KC : nullptr,
+                                        to_cache ? g + p.L.off_ks + tp * T::KS : nullptr);
                 } else {
                     const uint16_t* src = p.v_new + ((int64_t)b * H + h) * D;
                     quantize_row<KV, D>(src, p.rot_v, p.v_scale, st + off_vc + t * T::VC, st + off_vs + t * T::VS,
-                                        t, lane);
-                    if (hb == 0)
-                        quantize_row<KV, D>(src, p.rot_v, p.v_scale, g + p.L.off_vc + tp * T::VC,
-                                            g + p.L.off_vs + tp * T::VS, tp, lane);
+                                        t, lane, to_cache ? g + p.L.off_vc + tp * T::VC : nullptr,
+                                        to_cache ? g + p.L.off_vs + tp * T::VS : nullptr);
                 }
             }
             asm volatile("bar.sync 5, %0;" ::"r"(kDecThreads) : "memory");
@@ -943,6 +919,7 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
                 fin[tid] = M;
                 fin[8 + tid] = Ls;
             }
+#pragma unroll 1
             for (int w = 0; w < 4; w++) {
                 if (tw == w) {   // both halves write disjoint head_dim ranges
 #pragma unroll
@@ -1038,7 +1015,7 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
             if (seg_w0 >= w0 && seg_w0 + c.nspans <= w1) continue;     // whole: already stored
             const int i_first = part.owner(c.b, c.hh, 0);
             const int i_last = part.owner(c.b, c.hh, c.nspans - 1);
-            merge_segment<D>(p, c.b, c.h, c.hb, seg_w0, i_first, i_last, part, fin);
+            merge_segment<D>(p, c.b, c.h, c.hb, seg_w0, i_first, i_last, part);
         }
     }
 }
@@ -1109,10 +1086,11 @@ cudaError_t plan_decode(const Layout& L, int B, int HB, int max_seq_len, DecodeP
             if (stages < (ctas >= 2 ? 3 : 2)) continue;
             const int64_t stage_bytes = ((int64_t)stages * U.bytes + 127) & ~(int64_t)127;
             int64_t cap = (work + grid - 1) / grid + 1;                  // units of the largest range
+            if (cap < stages) cap = stages;   // the first stages' page ids go there too
             const int64_t room = kMinPids + (budget - (int64_t)fixed - stage_bytes) / 4;
             if (cap > room) cap = room;
             if (cap > 4096) cap = 4096;
-            const size_t smem = (size_t)stage_bytes + fixed + 4 * (size_t)(cap - kMinPids);
+            const size_t smem = (size_t)stage_bytes + (fixed - 4 * (size_t)kMinPids) + 4 * (size_t)cap;
             if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
                 return e;
             int resident = 0;

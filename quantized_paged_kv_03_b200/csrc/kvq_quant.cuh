@@ -7,7 +7,10 @@
 //   bf16 row -> [Hadamard-256] -> group amax -> scale rounded to its own format
 //   -> codes = round-nearest-even(value / decoded scale), saturating.
 // D/32 values per lane, a shuffle-based Hadamard, shuffle reductions for the
-// group amax, one store per lane through the row's chunk permutation.
+// group amax, one store per lane through the row's chunk permutation -- into
+// one row, or into two (the fused decode writes the same row into its stage
+// and into the cache; their row indices differ by a multiple of 64, so the
+// chunk permutation is the same).
 #pragma once
 
 #include "kvq_internal.h"
@@ -16,8 +19,8 @@ namespace kvq {
 
 template <int KIND, int D>
 __device__ __forceinline__ void quantize_row(const uint16_t* __restrict__ src, bool rot, float tscale,
-                                             uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
-                                             int t, int lane) {
+                                             uint8_t* codes, uint8_t* scales, int t, int lane,
+                                             uint8_t* codes2 = nullptr, uint8_t* scales2 = nullptr) {
     constexpr int EPL = D / 32;                 // values per lane
     constexpr int BITS = kind_bits(KIND);
     constexpr int BPL = EPL * BITS / 8;         // code bytes per lane
@@ -38,7 +41,7 @@ __device__ __forceinline__ void quantize_row(const uint16_t* __restrict__ src, b
     }
 
     const int swz = row_swizzle(KIND, D, t);
-    uint8_t* dst = codes + phys_byte(lane * BPL, swz);
+    const int lane_off = phys_byte(lane * BPL, swz);
     uint32_t out[4] = {0, 0, 0, 0};
 
     if constexpr (KIND == RK_BF16RAW) {
@@ -68,7 +71,10 @@ __device__ __forceinline__ void quantize_row(const uint16_t* __restrict__ src, b
             const float qmax = (KIND == RK_E4M3_ROW256) ? 448.f : 127.f;
             uint16_t sb = enc_f16_sat(__fdiv_rn(amax, qmax));
             float s = f16_bits_to_f32(sb);
-            if (leader) *reinterpret_cast<uint16_t*>(scales + 2 * g) = sb;
+            if (leader) {
+                *reinterpret_cast<uint16_t*>(scales + 2 * g) = sb;
+                if (scales2) *reinterpret_cast<uint16_t*>(scales2 + 2 * g) = sb;
+            }
             if constexpr (KIND == RK_E4M3_ROW256) {
 #pragma unroll
                 for (int i = 0; i < EPL / 2; i++) {
@@ -85,7 +91,10 @@ __device__ __forceinline__ void quantize_row(const uint16_t* __restrict__ src, b
         } else if constexpr (KIND == RK_E2M1_G16) {
             uint32_t sb = enc_e4m3x2(__fdiv_rn(amax, 6.f), 0.f) & 0x7Fu;    // UE4M3
             float s = e4m3_to_f32(sb);
-            if (leader) scales[g] = (uint8_t)sb;
+            if (leader) {
+                scales[g] = (uint8_t)sb;
+                if (scales2) scales2[g] = (uint8_t)sb;
+            }
 #pragma unroll
             for (int i = 0; i < EPL / 2; i++) {
                 uint32_t c = (s != 0.f) ? enc_e2m1x2(__fdiv_rn(x[2 * i], s), __fdiv_rn(x[2 * i + 1], s)) : 0u;
@@ -98,7 +107,10 @@ __device__ __forceinline__ void quantize_row(const uint16_t* __restrict__ src, b
             int E = min(127, max(-127, e2 - 1 - 8));
             float inv = (-E == -127) ? __uint_as_float(0x00400000u) : __uint_as_float((uint32_t)(127 - E) << 23);
             bool nz = amax > 0.f;
-            if (leader) scales[g] = nz ? (uint8_t)(E + 127) : (uint8_t)0;
+            if (leader) {
+                scales[g] = nz ? (uint8_t)(E + 127) : (uint8_t)0;
+                if (scales2) scales2[g] = scales[g];
+            }
 #pragma unroll
             for (int i = 0; i < EPL / 2; i++) {
                 uint32_t c = nz ? enc_e4m3x2(__fmul_rn(x[2 * i], inv), __fmul_rn(x[2 * i + 1], inv)) : 0u;
@@ -107,15 +119,19 @@ __device__ __forceinline__ void quantize_row(const uint16_t* __restrict__ src, b
         }
     }
     // store this lane's code bytes (a whole lane slice never straddles a 16-byte chunk)
-    if constexpr (BPL == 16) {
-        *reinterpret_cast<uint4*>(dst) = make_uint4(out[0], out[1], out[2], out[3]);
-    } else if constexpr (BPL == 8) {
-        *reinterpret_cast<uint2*>(dst) = make_uint2(out[0], out[1]);
-    } else if constexpr (BPL == 4) {
-        *reinterpret_cast<uint32_t*>(dst) = out[0];
-    } else {
-        *reinterpret_cast<uint16_t*>(dst) = (uint16_t)out[0];
-    }
+    auto store = [&](uint8_t* dst) {
+        if constexpr (BPL == 16) {
+            *reinterpret_cast<uint4*>(dst) = make_uint4(out[0], out[1], out[2], out[3]);
+        } else if constexpr (BPL == 8) {
+            *reinterpret_cast<uint2*>(dst) = make_uint2(out[0], out[1]);
+        } else if constexpr (BPL == 4) {
+            *reinterpret_cast<uint32_t*>(dst) = out[0];
+        } else {
+            *reinterpret_cast<uint16_t*>(dst) = (uint16_t)out[0];
+        }
+    };
+    store(codes + lane_off);
+    if (codes2) store(codes2 + lane_off);
 }
 
 }  // namespace kvq
