@@ -177,8 +177,37 @@ class Arm:
         self.ws = self.cache.workspace(w.B, w.Hq, w.max_seq_len)
         self.dec_bytes = decode_bytes(w, self.tb)
         self.app_bytes = append_bytes(w.B, w, self.tb)
+        self.qerr = self.quant_error()
         self.w.k = self.w.v = None     # host copies no longer needed
         torch.cuda.synchronize()
+
+    def quant_error(self, n_samples: int = 3):
+        """Quantisation error, for information: one fused step's outputs against
+        fp64 attention over the unquantised bf16 K/V (the values a BF16 cache
+        holds), on sampled (sequence, kv-head) pairs -- the shortest, the
+        longest and a middle-length sequence, kv-head 0 and the last kv-head."""
+        torch, w = self.torch, self.w
+        self.step()
+        out = self.out.double()
+        G = w.Hq // w.H
+        order = np.argsort(w.seq_lens, kind="stable")
+        seqs = sorted({int(order[0]), int(order[len(order) // 2]), int(order[-1])})[:n_samples]
+        bf16 = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda().view(
+            torch.bfloat16).double()
+        worst_max, worst_rms = 0.0, 0.0
+        for b in seqs:
+            rows = slice(int(w.starts[b]), int(w.starts[b + 1]))
+            for h in sorted({0, w.H - 1}):
+                k, v = bf16(w.k[rows, h]), bf16(w.v[rows, h])
+                q = bf16(w.q[b, h * G:(h + 1) * G])
+                ref = torch.softmax((q @ k.T) / np.sqrt(w.D), dim=-1) @ v
+                err = out[b, h * G:(h + 1) * G] - ref
+                worst_max = max(worst_max, float(err.abs().max() / v.abs().max()))
+                worst_rms = max(worst_rms, float(err.norm() / ref.norm()))
+                del k, v
+        return {"max_abs_over_max_abs_v": round(worst_max, 6), "rel_rms": round(worst_rms, 6),
+                "sample": f"sequences {seqs} (lengths {[int(w.seq_lens[b]) for b in seqs]}), "
+                          f"kv-heads {sorted({0, w.H - 1})}; reference: fp64 attention over the bf16 inputs"}
 
     def step(self):
         """One decode step, one launch: append each sequence's new token and attend."""
@@ -434,7 +463,8 @@ def main():
                     "tokens_per_s": round(a.w.B / (sm * 1e-3), 1),
                     "decode_only_ms": round(dm, 5),
                     "decode_only_GBps": round(a.dec_bytes / (dm * 1e-3) / 1e9, 1),
-                    "step_bytes": sb, "bytes_per_token_head": a.tb}
+                    "step_bytes": sb, "bytes_per_token_head": a.tb,
+                    "quant_error_vs_bf16": a.qerr}
                 del a
                 torch.cuda.empty_cache()
 
@@ -459,6 +489,7 @@ def main():
             "tokens_per_s": round(tokens, 1),
             "pct_of_peak": round(100 * value / peak, 2),
             "decode_only_GBps": round(dec_gbs, 1),
+            "quant_error_vs_bf16": arm.qerr,
             "roofline": {"bound": "hbm", "achieved": round(step_gbs, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(step_gbs / peak, 4), "traffic": headline_traffic(args.config, args.batch),
                          "traffic_unit": "bytes per launch (ncu dram read + write)",

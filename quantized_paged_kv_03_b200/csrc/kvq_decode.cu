@@ -404,7 +404,27 @@ __host__ __device__ constexpr int decode_ctas(int kk, int vk, int D) {
                : 2;
 }
 
+// The fused append (kvq_append_decode) of one sequence's newest token: warp 0
+// quantises its K row, warp 1 its V row, into the stage (row t of the unit)
+// and, when g is set, into the cache slab (row tp of the page).  Out of line:
+// it runs once per sequence, and keeping it out of the decode loop keeps the
+// loop's code compact.
 template <int KK, int KV, int D>
+__device__ __noinline__ void fused_append_rows(int warp, int lane, const uint16_t* k_src, const uint16_t* v_src,
+                                               bool rot_k, bool rot_v, float k_scale, float v_scale, uint8_t* st,
+                                               uint8_t* g, int t, int tp, int u_ks, int u_vc, int u_vs, int c_ks,
+                                               int c_vc, int c_vs) {
+    using T = DecTraits<KK, KV, D>;
+    if (warp == 0) {
+        quantize_row<KK, D>(k_src, rot_k, k_scale, st + t * T::KC, st + u_ks + t * T::KS, t, lane,
+                            g ? g + tp * T::KC : nullptr, g ? g + c_ks + tp * T::KS : nullptr);
+    } else {
+        quantize_row<KV, D>(v_src, rot_v, v_scale, st + u_vc + t * T::VC, st + u_vs + t * T::VS, t, lane,
+                            g ? g + c_vc + tp * T::VC : nullptr, g ? g + c_vs + tp * T::VS : nullptr);
+    }
+}
+
+template <int KK, int KV, int D, bool FUSED>
 __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_kernel(const DecodeParams p) {
     using T = DecTraits<KK, KV, D>;
     extern __shared__ __align__(128) uint8_t smem[];
@@ -684,7 +704,7 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
         // ---- this pair's 16-token tiles of the page
         const uint32_t stg = (uint32_t)s * (uint32_t)U.bytes;   // byte offset of the stage
 
-        if (p.k_new != nullptr && cc.span == cc.nspans - 1) {
+        if (FUSED && cc.span == cc.nspans - 1) {
             // fused append: the sequence's newest token (position seq_len - 1) lies
             // in its last unit.  Quantise it into this stage (row t of the unit),
             // over whatever the copy brought, and into the cache (row tp of the
@@ -694,20 +714,11 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
             const int tp = t + (cc.span & ((1 << U.lg_up) - 1)) * U.sp;
             if (warp < 2) {
                 const int pid = (i < p.pid_cap) ? pids[i] : page_id(w0 + i);
-                uint8_t* g = p.slabs + ((int64_t)pid * H + h) * slab;
-                uint8_t* st = smem + stg;
-                const bool to_cache = (hb == 0);
-                if (warp == 0) {
-                    const uint16_t* src = p.k_new + ((int64_t)b * H + h) * D;
-                    quantize_row<KK, D>(src, p.rot_k, p.k_scale, st + t * T::KC, st + off_ks + t * T::KS, t, lane,
-                                        to_cache ? g + tp * T::KC : nullptr,
-                                        to_cache ? g + p.L.off_ks + tp * T::KS : nullptr);
-                } else {
-                    const uint16_t* src = p.v_new + ((int64_t)b * H + h) * D;
-                    quantize_row<KV, D>(src, p.rot_v, p.v_scale, st + off_vc + t * T::VC, st + off_vs + t * T::VS,
-                                        t, lane, to_cache ? g + p.L.off_vc + tp * T::VC : nullptr,
-                                        to_cache ? g + p.L.off_vs + tp * T::VS : nullptr);
-                }
+                uint8_t* g = (hb == 0) ? p.slabs + ((int64_t)pid * H + h) * slab : nullptr;
+                const int64_t row = (int64_t)b * H + h;
+                fused_append_rows<KK, KV, D>(warp, lane, p.k_new + row * D, p.v_new + row * D, p.rot_k, p.rot_v,
+                                             p.k_scale, p.v_scale, smem + stg, g, t, tp, (int)off_ks, (int)off_vc,
+                                             (int)off_vs, (int)p.L.off_ks, (int)p.L.off_vc, (int)p.L.off_vs);
             }
             asm volatile("bar.sync 5, %0;" ::"r"(kDecThreads) : "memory");
         }
@@ -1023,16 +1034,17 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
 // ------------------------------------------------------------ host side
 
 template <int KK, int KV, int D>
-static const void* kernel_ptr() {
-    return reinterpret_cast<const void*>(&decode_kernel<KK, KV, D>);
+static const void* kernel_ptr(bool fused) {
+    return fused ? reinterpret_cast<const void*>(&decode_kernel<KK, KV, D, true>)
+                 : reinterpret_cast<const void*>(&decode_kernel<KK, KV, D, false>);
 }
 
-static const void* decode_kernel_for(int fmt, int D) {
+static const void* decode_kernel_for(int fmt, int D, bool fused) {
     const int kk = kind_of(fmt, 0), vk = kind_of(fmt, 1);
-#define KVQ_CASE(KK, KV)                                   \
-    if (kk == KK && vk == KV) {                            \
-        if (D == 256) return kernel_ptr<KK, KV, 256>();    \
-        if (D == 128) return kernel_ptr<KK, KV, 128>();    \
+#define KVQ_CASE(KK, KV)                                        \
+    if (kk == KK && vk == KV) {                                 \
+        if (D == 256) return kernel_ptr<KK, KV, 256>(fused);    \
+        if (D == 128) return kernel_ptr<KK, KV, 128>(fused);    \
     }
     KVQ_CASE(RK_BF16RAW, RK_FP16)
     KVQ_CASE(RK_E4M3_ROW256, RK_E4M3_ROW256)
@@ -1065,8 +1077,9 @@ cudaError_t plan_decode(const Layout& L, int B, int HB, int max_seq_len, DecodeP
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&smem_blk, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess) return e;
-    const void* kern = decode_kernel_for(L.fmt, L.D);
-    if (!kern) return cudaErrorInvalidValue;
+    // decode-only and fused kernels share the plan (and so the workspace size)
+    const void* kerns[2] = {decode_kernel_for(L.fmt, L.D, false), decode_kernel_for(L.fmt, L.D, true)};
+    if (!kerns[0] || !kerns[1]) return cudaErrorInvalidValue;
     // The most CTAs per SM the kernel allows, each with at least three stages
     // (one CTA: two).  A stage holds a whole page if that fits, else (128- and
     // 256-token pages) a 64-token unit.  The shared memory left over holds the
@@ -1091,12 +1104,18 @@ cudaError_t plan_decode(const Layout& L, int B, int HB, int max_seq_len, DecodeP
             if (cap > room) cap = room;
             if (cap > 4096) cap = 4096;
             const size_t smem = (size_t)stage_bytes + (fixed - 4 * (size_t)kMinPids) + 4 * (size_t)cap;
-            if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
-                return e;
-            int resident = 0;
-            if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident, kern, kDecThreads, smem)) != cudaSuccess)
-                return e;
-            if (resident < ctas) continue;
+            int fits = 1;
+            for (const void* kern : kerns) {
+                if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
+                    cudaSuccess)
+                    return e;
+                int resident = 0;
+                if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident, kern, kDecThreads, smem)) !=
+                    cudaSuccess)
+                    return e;
+                if (resident < ctas) fits = 0;
+            }
+            if (!fits) continue;
             plan->stages = (int)stages;
             plan->threads = kDecThreads;
             plan->pid_cap = (int)cap;
@@ -1127,7 +1146,7 @@ void decode_workspace_zero_region(const Layout& L, int B, int HB, int grid, size
 }
 
 cudaError_t launch_decode(const DecodeParams& p, const DecodePlan& plan, cudaStream_t s) {
-    const void* k = decode_kernel_for(p.L.fmt, p.L.D);
+    const void* k = decode_kernel_for(p.L.fmt, p.L.D, p.k_new != nullptr);
     if (!k) return cudaErrorInvalidValue;
     DecodeParams q = p;
     q.U = make_span(p.L, plan.lg_up);
