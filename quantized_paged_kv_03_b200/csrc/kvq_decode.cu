@@ -37,6 +37,10 @@
 namespace kvq {
 
 constexpr int kDecThreads = 256;   // 8 warps: 4 tile slots x 2 head_dim halves
+// Row stride (floats) of the output-combine buffer: 4 floats of padding per head
+// row spread the heads a warp writes over different banks.
+template <int D>
+constexpr int kOsmStride = D + 4;
 constexpr int kMaxStages = 8;
 constexpr int kMaxBatch = 4096;
 constexpr long kWaitPolls = 1l << 22;
@@ -275,16 +279,27 @@ struct Partition {
     }
 };
 
+// The Hadamard-256 of one row held 8 values per lane, out of line: the segment
+// start (rotating q) and the segment end (rotating the output back) share one
+// copy of the code, which keeps those rarely run paths short to fetch.
+struct Row8 {
+    float v[8];
+};
+__device__ __noinline__ Row8 fwht256_row(Row8 x, int lane) {
+    fwht256_warp(x.v, lane);
+    return x;
+}
+
 // Store EPL consecutive output values (fp32 or bf16) at element offset `ob`.
 template <int EPL>
-__device__ __forceinline__ void store_out(const DecodeParams& p, int64_t ob, const float* x) {
-    if (p.out_fp32) {
-        float* dst = reinterpret_cast<float*>(p.out) + ob;
+__device__ __forceinline__ void store_out(void* out, int out_fp32, int64_t ob, const float* x) {
+    if (out_fp32) {
+        float* dst = reinterpret_cast<float*>(out) + ob;
 #pragma unroll
         for (int e = 0; e < EPL; e += 4)
             *reinterpret_cast<float4*>(dst + e) = make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]);
     } else {
-        uint16_t* dst = reinterpret_cast<uint16_t*>(p.out) + ob;
+        uint16_t* dst = reinterpret_cast<uint16_t*>(out) + ob;
 #pragma unroll
         for (int e = 0; e < EPL; e += 4)
             *reinterpret_cast<uint2*>(dst + e) = make_uint2(pack_bf16(x[e], x[e + 1]), pack_bf16(x[e + 2], x[e + 3]));
@@ -330,12 +345,13 @@ __device__ __forceinline__ bool grid_barrier(unsigned* bar, unsigned G, int* fla
 // output's threads fold the parts in with a running (max, sum, output) -- the
 // log-sum-exp merge -- then combine their folds by shuffles; no block barrier.
 template <int D>
-__device__ __forceinline__ void merge_segment(const DecodeParams& p, int b, int h, int hb, int64_t seg_w0,
-                                              int i_first, int i_last, const Partition& part) {
+__device__ __forceinline__ void merge_segment(const float* partials, void* out, int out_fp32, float o_mult, int Hq,
+                                           int Gq, int b, int h, int hb, int64_t seg_w0, int i_first, int i_last,
+                                           Partition part) {
     const int tid = threadIdx.x;
     const int P = i_last - i_first + 1;
     const int j = (int)blockIdx.x - i_first;
-    const int gv = min(8, p.G - hb * 8);
+    const int gv = min(8, Gq - hb * 8);
     const int NU = gv * (D / 4);
     const int o0 = (int)((int64_t)j * NU / P), o1 = (int)((int64_t)(j + 1) * NU / P);
     const int no = o1 - o0;
@@ -352,7 +368,7 @@ __device__ __forceinline__ void merge_segment(const DecodeParams& p, int b, int 
         if (valid) {
             for (int k = pl; k < P; k += tpo) {
                 const int i = i_first + k;
-                const float* pk = p.partials + ((int64_t)i * 2 + (part.start(i) >= seg_w0 ? 0 : 1)) * (16 + 8 * D);
+                const float* pk = partials + ((int64_t)i * 2 + (part.start(i) >= seg_w0 ? 0 : 1)) * (16 + 8 * D);
                 const float mk = __ldcg(pk + g), lk = __ldcg(pk + 8 + g);
                 const float4 v = __ldcg(reinterpret_cast<const float4*>(pk + 16 + g * D) + d4);
                 if (mk == -INFINITY) continue;
@@ -376,10 +392,10 @@ __device__ __forceinline__ void merge_segment(const DecodeParams& p, int b, int 
             M = Mn;
         }
         if (valid && pl == 0) {
-            const float inv = (L > 0.f) ? p.o_mult / L : 0.f;
+            const float inv = (L > 0.f) ? o_mult / L : 0.f;
             const float x[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
-            const int64_t oo = ((int64_t)b * p.Hq + h * p.G + hb * 8 + g) * D + 4 * d4;
-            store_out<4>(p, oo, x);
+            const int64_t oo = ((int64_t)b * Hq + h * Gq + hb * 8 + g) * D + 4 * d4;
+            store_out<4>(out, out_fp32, oo, x);
         }
     }
 }
@@ -445,7 +461,7 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
     Producer* prod = reinterpret_cast<Producer*>(smem + off);
     off += 32;
     float* osm = reinterpret_cast<float*>(smem + off);   // [8][D]: q staging / output combine / score exchange
-    off += (8 * D * 4 > 8192 ? 8 * D * 4 : 8192);
+    off += (8 * kOsmStride<D> * 4 > 8192 ? 8 * kOsmStride<D> * 4 : 8192);
     float4* xbuf = reinterpret_cast<float4*>(osm);       // [2 parity][4 tiles][2 halves][32 lanes]
     uint8_t* qst = smem + off;                           // q fragments of the segment (fp16 / bf16 hi, lo)
     off += 8 * (size_t)D * 2 * T::QS;
@@ -652,7 +668,14 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
 #pragma unroll
                     for (int e = 0; e < T::EPL; e++) x[e] = bf16_bits_to_f32((raw[e >> 1] >> ((e & 1) * 16)) & 0xFFFFu);
                     if constexpr (D == 256) {
-                        if (p.rot_k) fwht256_warp(x, lane);
+                        if (p.rot_k) {
+                            Row8 y;
+#pragma unroll
+                            for (int e = 0; e < 8; e++) y.v[e] = x[e];
+                            y = fwht256_row(y, lane);
+#pragma unroll
+                            for (int e = 0; e < 8; e++) x[e] = y.v[e];
+                        }
                     }
 #pragma unroll
                     for (int e = 0; e < T::EPL; e++) x[e] *= p.q_mult;
@@ -905,6 +928,8 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
                 l1 += __shfl_xor_sync(0xffffffffu, l1, m);
             }
             __syncthreads();   // all tiles of the segment done; osm free
+            for (int k = tid; k < 2 * kOsmStride<D>; k += kDecThreads)
+                reinterpret_cast<float4*>(osm)[k] = make_float4(0.f, 0.f, 0.f, 0.f);
             if (hf == 0 && r == 0) {
                 wml[tw * 16 + 2 * j] = m0;
                 wml[tw * 16 + 2 * j + 1] = m1;
@@ -930,31 +955,23 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
                 fin[tid] = M;
                 fin[8 + tid] = Ls;
             }
+            {
+                // this lane's outputs: heads 2j, 2j+1; dims (relative to its half)
+                // VCW*(ul/VCH) + 4*(ul%VCH) + [0 | 2] + lane part
+                float* pa = osm + (2 * j) * kOsmStride<D> + hf * (D / 2) + 4 * T::VCH * (r >> 1) + (r & 1);
+                float* pb = pa + kOsmStride<D>;
 #pragma unroll 1
-            for (int w = 0; w < 4; w++) {
-                if (tw == w) {   // both halves write disjoint head_dim ranges
+                for (int w = 0; w < 4; w++) {
+                    if (tw == w) {   // both halves write disjoint head_dim ranges
 #pragma unroll
-                    for (int ul = 0; ul < T::DTILES / 2; ul++) {
-                        const int u = hf * (T::DTILES / 2) + ul;
-                        const int c = u / T::VCH, uu = u % T::VCH;
-                        const int base = T::VCW * c + 4 * uu;
-                        const int da = base + 4 * T::VCH * (r >> 1) + (r & 1);   // logical row r
-                        const int db = da + 2;                                    // logical row r + 8
-                        // head n's row is stored with d ^ (n << 2), which spreads the
-                        // four heads a warp writes over different banks
-                        float* oa0 = osm + (2 * j) * D;
-                        float* oa1 = osm + (2 * j + 1) * D;
-                        const int x0 = (2 * j) << 2, x1 = (2 * j + 1) << 2;
-                        if (w == 0) {
-                            oa0[da ^ x0] = o[ul][0] * f0; oa1[da ^ x1] = o[ul][1] * f1;
-                            oa0[db ^ x0] = o[ul][2] * f0; oa1[db ^ x1] = o[ul][3] * f1;
-                        } else {
-                            oa0[da ^ x0] += o[ul][0] * f0; oa1[da ^ x1] += o[ul][1] * f1;
-                            oa0[db ^ x0] += o[ul][2] * f0; oa1[db ^ x1] += o[ul][3] * f1;
+                        for (int ul = 0; ul < T::DTILES / 2; ul++) {
+                            const int d = T::VCW * (ul / T::VCH) + 4 * (ul % T::VCH);
+                            pa[d] += o[ul][0] * f0; pb[d] += o[ul][1] * f1;
+                            pa[d + 2] += o[ul][2] * f0; pb[d + 2] += o[ul][3] * f1;
                         }
                     }
+                    __syncthreads();
                 }
-                __syncthreads();
             }
 
             // ---- a whole segment is normalised and stored here; a segment cut by
@@ -973,9 +990,16 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
                     const float inv = whole ? ((Ls > 0.f) ? p.o_mult / Ls : 0.f) : 1.f;
                     float x[8];
 #pragma unroll
-                    for (int e = 0; e < T::EPL; e++) x[e] = osm[nh * D + ((lane * T::EPL + e) ^ (nh << 2))] * inv;
+                    for (int e = 0; e < T::EPL; e++) x[e] = osm[nh * kOsmStride<D> + lane * T::EPL + e] * inv;
                     if constexpr (D == 256) {
-                        if (p.rot_v) fwht256_warp(x, lane);
+                        if (p.rot_v) {
+                            Row8 y;
+#pragma unroll
+                            for (int e = 0; e < 8; e++) y.v[e] = x[e];
+                            y = fwht256_row(y, lane);
+#pragma unroll
+                            for (int e = 0; e < 8; e++) x[e] = y.v[e];
+                        }
                     }
                     if (!whole) {
                         float* dst = part + 16 + nh * D + lane * T::EPL;
@@ -984,7 +1008,7 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
                             *reinterpret_cast<float4*>(dst + e) = make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]);
                     } else {
                         const int64_t ob = ((int64_t)b * p.Hq + h * p.G + gq) * D + lane * T::EPL;
-                        store_out<T::EPL>(p, ob, x);
+                        store_out<T::EPL>(p.out, p.out_fp32, ob, x);
                     }
                 }
             }
@@ -1026,7 +1050,8 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
             if (seg_w0 >= w0 && seg_w0 + c.nspans <= w1) continue;     // whole: already stored
             const int i_first = part.owner(c.b, c.hh, 0);
             const int i_last = part.owner(c.b, c.hh, c.nspans - 1);
-            merge_segment<D>(p, c.b, c.h, c.hb, seg_w0, i_first, i_last, part);
+            merge_segment<D>(p.partials, p.out, p.out_fp32, p.o_mult, p.Hq, p.G, c.b, c.h, c.hb, seg_w0, i_first,
+                             i_last, part);
         }
     }
 }
@@ -1063,7 +1088,8 @@ bool decode_supported(int fmt, int D) {
 }
 
 static size_t fixed_smem(int D, int B, int pid_cap, int qs) {
-    const size_t osm = 8 * (size_t)D * 4 > 8192 ? 8 * (size_t)D * 4 : 8192;
+    const size_t ostr = (size_t)D + 4;   // kOsmStride
+    const size_t osm = 8 * ostr * 4 > 8192 ? 8 * ostr * 4 : 8192;
     const size_t qst = 8 * (size_t)D * 2 * qs;
     return 8 * kMaxStages + 4 * kMaxStages + 32 + osm + qst + 4 * 16 * 4 + 16 * 4 + 16 + 4 * (size_t)(B + 1) +
            4 * (size_t)pid_cap + 128;
