@@ -344,6 +344,8 @@ __device__ __forceinline__ bool grid_barrier(unsigned* bar, unsigned G, int* fla
 // produces float4 outputs [o0, o1) of the segment's gv x D/4.  One pass: each
 // output's threads fold the parts in with a running (max, sum, output) -- the
 // log-sum-exp merge -- then combine their folds by shuffles; no block barrier.
+constexpr int kMergeBatch = 2;
+
 template <int D>
 __device__ __forceinline__ void merge_segment(const float* partials, void* out, int out_fp32, float o_mult, int Hq,
                                            int Gq, int b, int h, int hb, int64_t seg_w0, int i_first, int i_last,
@@ -356,6 +358,9 @@ __device__ __forceinline__ void merge_segment(const float* partials, void* out, 
     const int o0 = (int)((int64_t)j * NU / P), o1 = (int)((int64_t)(j + 1) * NU / P);
     const int no = o1 - o0;
     if (no <= 0) return;
+    // The segment is the first of every part's range except possibly the first
+    // part's (slot 0 holds a range's first segment, slot 1 its last).
+    const int slot0 = part.start(i_first) >= seg_w0 ? 0 : 1;
     int tpo = 1;   // threads per output, splitting the parts
     while (tpo < 16 && tpo * 2 * no <= kDecThreads) tpo *= 2;
     const int per_pass = kDecThreads / tpo;
@@ -366,18 +371,31 @@ __device__ __forceinline__ void merge_segment(const float* partials, void* out, 
         float M = -INFINITY, L = 0.f;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         if (valid) {
-            for (int k = pl; k < P; k += tpo) {
-                const int i = i_first + k;
-                const float* pk = partials + ((int64_t)i * 2 + (part.start(i) >= seg_w0 ? 0 : 1)) * (16 + 8 * D);
-                const float mk = __ldcg(pk + g), lk = __ldcg(pk + 8 + g);
-                const float4 v = __ldcg(reinterpret_cast<const float4*>(pk + 16 + g * D) + d4);
-                if (mk == -INFINITY) continue;
-                const float Mn = fmaxf(M, mk);
-                const float a = (M == -INFINITY) ? 0.f : exp2f(M - Mn), w = exp2f(mk - Mn);
-                acc.x = fmaf(w, v.x, acc.x * a); acc.y = fmaf(w, v.y, acc.y * a);
-                acc.z = fmaf(w, v.z, acc.z * a); acc.w = fmaf(w, v.w, acc.w * a);
-                L = fmaf(w, lk, L * a);
-                M = Mn;
+            // parts in groups of kMergeBatch, all loads of a group in flight together
+            for (int k0 = pl; k0 < P; k0 += kMergeBatch * tpo) {
+                float mk[kMergeBatch], lk[kMergeBatch];
+                float4 v[kMergeBatch];
+#pragma unroll
+                for (int q = 0; q < kMergeBatch; q++) {
+                    const int k = k0 + q * tpo;
+                    mk[q] = -INFINITY;
+                    if (k < P) {
+                        const float* pk = partials + ((int64_t)(i_first + k) * 2 + (k == 0 ? slot0 : 0)) * (16 + 8 * D);
+                        mk[q] = __ldcg(pk + g);
+                        lk[q] = __ldcg(pk + 8 + g);
+                        v[q] = __ldcg(reinterpret_cast<const float4*>(pk + 16 + g * D) + d4);
+                    }
+                }
+#pragma unroll
+                for (int q = 0; q < kMergeBatch; q++) {
+                    if (mk[q] == -INFINITY) continue;
+                    const float Mn = fmaxf(M, mk[q]);
+                    const float a = (M == -INFINITY) ? 0.f : exp2f(M - Mn), w = exp2f(mk[q] - Mn);
+                    acc.x = fmaf(w, v[q].x, acc.x * a); acc.y = fmaf(w, v[q].y, acc.y * a);
+                    acc.z = fmaf(w, v[q].z, acc.z * a); acc.w = fmaf(w, v[q].w, acc.w * a);
+                    L = fmaf(w, lk[q], L * a);
+                    M = Mn;
+                }
             }
         }
         for (int m = 1; m < tpo; m <<= 1) {
