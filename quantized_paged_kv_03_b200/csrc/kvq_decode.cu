@@ -362,7 +362,7 @@ __device__ __forceinline__ void merge_segment(const float* partials, void* out, 
     // part's (slot 0 holds a range's first segment, slot 1 its last).
     const int slot0 = part.start(i_first) >= seg_w0 ? 0 : 1;
     int tpo = 1;   // threads per output, splitting the parts
-    while (tpo < 16 && tpo * 2 * no <= kDecThreads) tpo *= 2;
+    while (tpo < 32 && tpo * 2 * no <= kDecThreads) tpo *= 2;
     const int per_pass = kDecThreads / tpo;
     for (int ob = o0; ob < o1; ob += per_pass) {
         const int o = ob + tid / tpo, pl = tid % tpo;
