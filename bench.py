@@ -164,6 +164,13 @@ class Arm:
         for i in range(0, len(sp), step):     # bulk prefill, untimed
             self.cache.append(0, dev(kp[i:i + step]).view(torch.bfloat16),
                               dev(vp[i:i + step]).view(torch.bfloat16), dev(sp[i:i + step]))
+        # a bulk append to time on its own: the prefix's first rows again (same
+        # slots, same codes), at most 2^18 tokens
+        na = min(len(sp), 1 << 18)
+        self.app_k = dev(kp[:na]).view(torch.bfloat16)
+        self.app_v = dev(vp[:na]).view(torch.bfloat16)
+        self.app_s = dev(sp[:na])
+        self.bulk_tokens = na
         del kp, vp
         kn, vn, sn = w.new_tokens()
         self.h_k, self.h_v, self.h_s = kn, vn, sn
@@ -177,6 +184,7 @@ class Arm:
         self.ws = self.cache.workspace(w.B, w.Hq, w.max_seq_len)
         self.dec_bytes = decode_bytes(w, self.tb)
         self.app_bytes = append_bytes(w.B, w, self.tb)
+        self.bulk_bytes = append_bytes(self.bulk_tokens, w, self.tb)
         self.qerr = self.quant_error()
         self.w.k = self.w.v = None     # host copies no longer needed
         torch.cuda.synchronize()
@@ -213,6 +221,9 @@ class Arm:
         """One decode step, one launch: append each sequence's new token and attend."""
         self.cache.append_decode(0, self.k_new, self.v_new, self.q, self.bt, self.sl, self.w.max_seq_len,
                                  out=self.out, workspace=self.ws)
+
+    def bulk_append(self):
+        self.cache.append(0, self.app_k, self.app_v, self.app_s)
 
     def decode_only(self):
         self.cache.decode_attention(0, self.q, self.bt, self.sl, self.w.max_seq_len, out=self.out,
@@ -436,6 +447,7 @@ def main():
         dist.barrier()
     t_wall = time.perf_counter() - t_wall
     dec_t = arm.run(args.steps, args.warmup, flush, fn=arm.decode_only)
+    app_ms = max_over_ranks(float(arm.run(args.steps, args.warmup, flush, fn=arm.bulk_append).mean()), dist)
     step_ms = float(step_t.mean())
     step_bytes = arm.dec_bytes + arm.app_bytes
     bytes_per_s, step_ms_max = whole_job_rate(step_bytes, step_ms, dist)
@@ -456,6 +468,7 @@ def main():
                 a = Arm(cfg, f, seed_offset=rank)
                 sm = max_over_ranks(float(a.run(args.steps, args.warmup, flush).mean()), dist)
                 dm = max_over_ranks(float(a.run(args.steps, args.warmup, flush, fn=a.decode_only).mean()), dist)
+                am = max_over_ranks(float(a.run(args.steps, args.warmup, flush, fn=a.bulk_append).mean()), dist)
                 sb = a.dec_bytes + a.app_bytes
                 formats[f"{I.CONFIGS[cfg].name}/{f}"] = {
                     "step_ms": round(sm, 5), "step_GBps": round(sb / (sm * 1e-3) / 1e9, 1),
@@ -464,6 +477,10 @@ def main():
                     "decode_only_ms": round(dm, 5),
                     "decode_only_GBps": round(a.dec_bytes / (dm * 1e-3) / 1e9, 1),
                     "step_bytes": sb, "bytes_per_token_head": a.tb,
+                    "append_tokens": a.bulk_tokens, "append_ms": round(am, 5),
+                    "append_GBps": round(a.bulk_bytes / (am * 1e-3) / 1e9, 1),
+                    "append_pct_of_peak": round(100 * a.bulk_bytes / (am * 1e-3) / 1e9 / peak, 1),
+                    "append_tokens_per_s": round(a.bulk_tokens / (am * 1e-3), 1),
                     "quant_error_vs_bf16": a.qerr}
                 del a
                 torch.cuda.empty_cache()
@@ -490,6 +507,11 @@ def main():
             "pct_of_peak": round(100 * value / peak, 2),
             "decode_only_GBps": round(dec_gbs, 1),
             "quant_error_vs_bf16": arm.qerr,
+            "append": {"tokens": arm.bulk_tokens, "ms": round(app_ms, 5),
+                       "GBps": round(arm.bulk_bytes / (app_ms * 1e-3) / 1e9, 1),
+                       "pct_of_peak": round(100 * arm.bulk_bytes / (app_ms * 1e-3) / 1e9 / peak, 1),
+                       "tokens_per_s": round(arm.bulk_tokens / (app_ms * 1e-3), 1),
+                       "what": "bulk append of the prefix's first tokens (append_kernel alone)"},
             "roofline": {"bound": "hbm", "achieved": round(step_gbs, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(step_gbs / peak, 4), "traffic": headline_traffic(args.config, args.batch),
                          "traffic_unit": "bytes per launch (ncu dram read + write)",
