@@ -9,38 +9,67 @@
 //   bf16 row -> [Hadamard-256] -> group amax -> scale rounded to its own format
 //   -> codes = round-nearest-even(value / decoded scale), saturating -> 16-byte
 //   aligned stores into the slot's page slab.
-// One warp owns one (token, kv-head, K|V) row (quantize_row in kvq_quant.cuh).
+// One warp owns kAppendRows consecutive (token, kv-head, K|V) rows, loading
+// all of them before quantising each (quantize_loaded in kvq_quant.cuh).
 #include "kvq_quant.cuh"
 
 namespace kvq {
 
 // -------------------------------------------------------------- append
 
+constexpr int kAppendRows = 2;   // rows per warp, their loads in flight together
+
+// Row and slot arithmetic in 32 bits (64-bit division is a long software
+// sequence): the launch guarantees rows < 2^31; a slot below the pool capacity
+// fits 32 bits whenever the capacity does (`p.cap32`), else 64-bit division.
 template <int KK, int KV, int D>
 __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
     const int lane = threadIdx.x & 31;
-    const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);   // ((token*2 + kv)*H + h)
-    if (row >= (int64_t)p.n_tokens * 2 * p.L.H) return;
-    const int h = (int)(row % p.L.H);
-    const int kv = (int)((row / p.L.H) & 1);
-    const int64_t tok = row / (2 * p.L.H);
-    const int64_t slot = p.slots[tok];
-    if (slot < 0) return;
-    const int64_t cap = (int64_t)p.L.num_pages * p.L.P;
-    if (slot >= cap) {
-        if (lane == 0) atomicOr(p.status, kStatusBadSlot);
-        return;
+    const uint32_t H = (uint32_t)p.L.H;
+    const uint32_t nrows = (uint32_t)p.n_tokens * 2u * H;   // row = (token*2 + kv)*H + h
+    const uint32_t row0 = ((uint32_t)blockIdx.x * 8u + (threadIdx.x >> 5)) * kAppendRows;
+    RowBits raw[kAppendRows];
+    int64_t slot[kAppendRows];
+#pragma unroll
+    for (int r = 0; r < kAppendRows; r++) {
+        const uint32_t row = row0 + r;
+        slot[r] = -1;
+        if (row < nrows) {
+            const uint32_t hk = row / H;                 // token*2 + kv
+            const uint32_t h = row - hk * H, tok = hk >> 1;
+            slot[r] = p.slots[tok];
+            raw[r] = load_row<D>(((hk & 1) ? p.v : p.k) + ((int64_t)tok * H + h) * D, lane);
+        }
     }
-    const int64_t page = slot / p.L.P;
-    const int t = (int)(slot % p.L.P);
-    uint8_t* slab = p.slabs + (page * p.L.H + h) * p.L.slab;
-    const uint16_t* src = (kv ? p.v : p.k) + (tok * p.L.H + h) * D;
-    if (kv == 0) {
-        quantize_row<KK, D>(src, p.rot_k, p.k_scale, slab + (int64_t)t * p.L.kc, slab + p.L.off_ks + (int64_t)t * p.L.ks,
-                            t, lane);
-    } else {
-        quantize_row<KV, D>(src, p.rot_v, p.v_scale, slab + p.L.off_vc + (int64_t)t * p.L.vc,
-                            slab + p.L.off_vs + (int64_t)t * p.L.vs, t, lane);
+    const int64_t cap = (int64_t)p.L.num_pages * p.L.P;
+#pragma unroll
+    for (int r = 0; r < kAppendRows; r++) {
+        const uint32_t row = row0 + r;
+        if (slot[r] < 0) continue;   // past the end, or skipped by the caller
+        if (slot[r] >= cap) {
+            if (lane == 0) atomicOr(p.status, kStatusBadSlot);
+            continue;
+        }
+        const uint32_t hk = row / H;
+        const int h = (int)(row - hk * H), kv = (int)(hk & 1);
+        int64_t page;
+        int t;
+        if (p.cap32) {
+            const uint32_t sl = (uint32_t)slot[r], pg = sl / (uint32_t)p.L.P;
+            page = pg;
+            t = (int)(sl - pg * (uint32_t)p.L.P);
+        } else {
+            page = slot[r] / p.L.P;
+            t = (int)(slot[r] % p.L.P);
+        }
+        uint8_t* slab = p.slabs + (page * p.L.H + h) * p.L.slab;
+        if (kv == 0) {
+            quantize_loaded<KK, D>(raw[r], p.rot_k, p.k_scale, slab + (int64_t)t * p.L.kc,
+                                   slab + p.L.off_ks + (int64_t)t * p.L.ks, t, lane);
+        } else {
+            quantize_loaded<KV, D>(raw[r], p.rot_v, p.v_scale, slab + p.L.off_vc + (int64_t)t * p.L.vc,
+                                   slab + p.L.off_vs + (int64_t)t * p.L.vs, t, lane);
+        }
     }
 }
 
@@ -150,12 +179,24 @@ __global__ void encode_kernel(int code, const float* __restrict__ x, int64_t n, 
 // -------------------------------------------------------------- launchers
 
 template <int KK, int KV>
-static cudaError_t launch_append_kv(const AppendParams& p, cudaStream_t s) {
-    int64_t rows = (int64_t)p.n_tokens * 2 * p.L.H;
-    dim3 grid((unsigned)((rows + 7) / 8));
-    if (p.L.D == 256) append_kernel<KK, KV, 256><<<grid, 256, 0, s>>>(p);
-    else append_kernel<KK, KV, 128><<<grid, 256, 0, s>>>(p);
-    return cudaGetLastError();
+static cudaError_t launch_append_kv(const AppendParams& p0, cudaStream_t s) {
+    // launches of at most 2^30 rows (the kernel's row arithmetic is 32-bit)
+    AppendParams p = p0;
+    p.cap32 = (int64_t)p.L.num_pages * p.L.P < ((int64_t)1 << 31);
+    const int64_t per = ((int64_t)1 << 30) / (2 * p.L.H);
+    for (int64_t t0 = 0; t0 < p0.n_tokens; t0 += per) {
+        p.n_tokens = (int)(p0.n_tokens - t0 < per ? p0.n_tokens - t0 : per);
+        p.k = p0.k + t0 * p.L.H * p.L.D;
+        p.v = p0.v + t0 * p.L.H * p.L.D;
+        p.slots = p0.slots + t0;
+        const int64_t rows = (int64_t)p.n_tokens * 2 * p.L.H;
+        dim3 grid((unsigned)((rows + 8 * kAppendRows - 1) / (8 * kAppendRows)));
+        if (p.L.D == 256) append_kernel<KK, KV, 256><<<grid, 256, 0, s>>>(p);
+        else append_kernel<KK, KV, 128><<<grid, 256, 0, s>>>(p);
+        const cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s) {

@@ -15,6 +15,7 @@ struct AppendParams {
     bool rot_k, rot_v;
     float k_scale, v_scale;      // per-tensor scales (FP8_TENSOR)
     uint32_t* status;
+    bool cap32;                  // set by the launch: pool slots fit 31 bits
 };
 
 struct ReadParams {

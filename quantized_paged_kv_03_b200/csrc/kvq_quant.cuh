@@ -17,23 +17,32 @@
 
 namespace kvq {
 
+// A lane's D/32 bf16 values of one row (16 B for D=256, 8 B for D=128).
+struct RowBits {
+    uint32_t w[4];
+};
+template <int D>
+__device__ __forceinline__ RowBits load_row(const uint16_t* __restrict__ src, int lane) {
+    RowBits r;
+    if constexpr (D / 32 == 8) {
+        const uint4 v = *reinterpret_cast<const uint4*>(src + lane * 8);
+        r.w[0] = v.x; r.w[1] = v.y; r.w[2] = v.z; r.w[3] = v.w;
+    } else {
+        const uint2 v = *reinterpret_cast<const uint2*>(src + lane * 4);
+        r.w[0] = v.x; r.w[1] = v.y; r.w[2] = 0; r.w[3] = 0;
+    }
+    return r;
+}
+
 template <int KIND, int D>
-__device__ __forceinline__ void quantize_row(const uint16_t* __restrict__ src, bool rot, float tscale,
-                                             uint8_t* codes, uint8_t* scales, int t, int lane,
-                                             uint8_t* codes2 = nullptr, uint8_t* scales2 = nullptr) {
+__device__ __forceinline__ void quantize_loaded(const RowBits& rb, bool rot, float tscale, uint8_t* codes,
+                                                uint8_t* scales, int t, int lane, uint8_t* codes2 = nullptr,
+                                                uint8_t* scales2 = nullptr) {
     constexpr int EPL = D / 32;                 // values per lane
     constexpr int BITS = kind_bits(KIND);
     constexpr int BPL = EPL * BITS / 8;         // code bytes per lane
     float x[8];
-    uint32_t raw[4];
-    // load EPL bf16 values (16 B for D=256, 8 B for D=128)
-    if constexpr (EPL == 8) {
-        uint4 v = *reinterpret_cast<const uint4*>(src + lane * 8);
-        raw[0] = v.x; raw[1] = v.y; raw[2] = v.z; raw[3] = v.w;
-    } else {
-        uint2 v = *reinterpret_cast<const uint2*>(src + lane * 4);
-        raw[0] = v.x; raw[1] = v.y; raw[2] = 0; raw[3] = 0;
-    }
+    const uint32_t* raw = rb.w;
 #pragma unroll
     for (int e = 0; e < EPL; e++) x[e] = bf16_bits_to_f32((raw[e >> 1] >> ((e & 1) * 16)) & 0xFFFFu);
     if constexpr (EPL == 8) {
@@ -132,6 +141,13 @@ __device__ __forceinline__ void quantize_row(const uint16_t* __restrict__ src, b
     };
     store(codes + lane_off);
     if (codes2) store(codes2 + lane_off);
+}
+
+template <int KIND, int D>
+__device__ __forceinline__ void quantize_row(const uint16_t* __restrict__ src, bool rot, float tscale,
+                                             uint8_t* codes, uint8_t* scales, int t, int lane,
+                                             uint8_t* codes2 = nullptr, uint8_t* scales2 = nullptr) {
+    quantize_loaded<KIND, D>(load_row<D>(src, lane), rot, tscale, codes, scales, t, lane, codes2, scales2);
 }
 
 }  // namespace kvq
