@@ -170,7 +170,7 @@ __global__ void encode_kernel(int code, const float* __restrict__ x, int64_t n, 
     case 0: out[i] = (uint8_t)enc_e4m3x2(v, 0.f); break;
     case 1: out[i] = (uint8_t)(enc_e2m1x2(v, 0.f) & 0xF); break;
     case 2: out[i] = (uint8_t)(enc_int8(v) & 0xFF); break;
-    case 3: reinterpret_cast<uint16_t*>(out)[i] = enc_f16_sat(v); break;
+    case 3: reinterpret_cast<uint16_t*>(out)[i] = (uint16_t)(enc_f16x2_sat(v, 0.f) & 0xFFFFu); break;
     case 4: out[i] = (uint8_t)(enc_e4m3x2(v, 0.f) & 0x7F); break;
     default: break;
     }

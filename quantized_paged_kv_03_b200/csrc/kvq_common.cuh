@@ -142,6 +142,14 @@ __device__ __forceinline__ uint16_t enc_f16_sat(float x) {
     return b;
 }
 
+// two fp16 codes (RNE, saturating to +-65504), `lo` in bits 0..15: one
+// instruction for the pair; same results as enc_f16_sat on each value
+__device__ __forceinline__ uint32_t enc_f16x2_sat(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
 // two E4M3 codes, `lo` in bits 0..7
 __device__ __forceinline__ uint32_t enc_e4m3x2(float lo, float hi) {
     uint16_t r;

@@ -58,7 +58,7 @@ __device__ __forceinline__ void quantize_loaded(const RowBits& rb, bool rot, flo
         for (int i = 0; i < EPL / 2; i++) out[i] = raw[i];
     } else if constexpr (KIND == RK_FP16) {
 #pragma unroll
-        for (int i = 0; i < EPL / 2; i++) out[i] = enc_f16_sat(x[2 * i]) | ((uint32_t)enc_f16_sat(x[2 * i + 1]) << 16);
+        for (int i = 0; i < EPL / 2; i++) out[i] = enc_f16x2_sat(x[2 * i], x[2 * i + 1]);
     } else if constexpr (KIND == RK_E4M3_TENSOR) {
         // [FP8-KV]: one symmetric scale for the whole tensor; [TokenSpeed] unit scale = 1
 #pragma unroll
