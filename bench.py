@@ -19,6 +19,7 @@ import json
 import os
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -434,8 +435,7 @@ def main():
     spec = I.CONFIGS[args.config]
     fmt = args.format or spec.formats[0]
     arm = Arm(args.config, fmt, seed_offset=rank, batch=args.batch)
-    clocks_path = os.path.join(ROOT, "gpurun_out", f"bench_clocks_r{rank}.csv")
-    os.makedirs(os.path.dirname(clocks_path), exist_ok=True)
+    clocks_path = os.path.join(tempfile.gettempdir(), f"kvq_bench_clocks_{os.getpid()}_r{rank}.csv")
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
