@@ -8,15 +8,19 @@
 // not arithmetic) make this a streaming kernel: its roofline is HBM bandwidth.
 //
 // Design (B200, sm_100a):
-//  * Persistent cooperative grid, 8 warps per CTA.  The page-heads of the whole
-//    batch, ordered (sequence, kv-head, 8-head block, page), are cut into
-//    gridDim.x contiguous equal ranges, so ragged batches balance to within
-//    one page.
-//  * Each page slab (K codes, K scales, V codes, V scales of one kv-head: one
-//    contiguous range in HBM) arrives with ONE cp.async.bulk into a shared-memory
-//    stage, completion tracked by an mbarrier.  Warps release a stage with a
+//  * Persistent cooperative grid, 8 warps per CTA (three CTAs per SM where a
+//    64-token unit is small enough, else two).  The work units of the whole
+//    batch -- a page of one kv-head, or a 64-token span of a larger page --
+//    ordered (sequence, kv-head, 8-head block, unit), are cut into gridDim.x
+//    contiguous ranges of equal cost, where a unit costs 1 and every segment a
+//    range touches adds the fixed price of its start and end; ragged batches
+//    balance to within about one unit.
+//  * A whole-page unit (K codes, K scales, V codes, V scales of one kv-head:
+//    one contiguous range in HBM) arrives with ONE cp.async.bulk into a
+//    shared-memory stage; a span of a larger page with one copy per part.
+//    Completion is tracked by an mbarrier.  Warps release a stage with a
 //    shared counter; the last warp to release it issues the next copy into it,
-//    so warps never wait for each other page by page.
+//    so warps never wait for each other unit by unit.
 //  * A 16-token tile is owned by a warp pair: each warp takes one half of
 //    head_dim.  Codes become fp16 (exact for every format) in registers straight
 //    from shared memory and feed mma.sync m16n8k16 with the GQA group (<= 8
