@@ -326,6 +326,51 @@ class PagedCache:
         return out
 
 
+    def prefill(self, q_bf16: np.ndarray, cu_q_lens: np.ndarray, block_table: np.ndarray,
+                seq_lens: np.ndarray, scale: float | None = None, threads: int = 1) -> np.ndarray:
+        """Causal attention of a chunk of query tokens per sequence over the
+        cache (the multi-token form of the attention over the quantized pages,
+        [NInfer] "causal_cache"), plain definition:
+          q [Tq, Hq, D] bf16 bits; rows cu_q_lens[b] .. cu_q_lens[b+1]-1 are the
+          n_b query tokens of sequence b, in order.  Query token i of sequence b
+          sits at position pos = seq_lens[b] - n_b + i (the chunk is the last n_b
+          tokens of the sequence) and attends the cached tokens [0, pos], the
+          token itself included; query head h reads kv-head h // (Hq / H_kv).
+          A row with pos < 0 has no keys: its output is zero.
+        Returns out [Tq, Hq, D] fp64."""
+        Tq, Hq, D = q_bf16.shape
+        G = Hq // self.H
+        cu = np.asarray(cu_q_lens, np.int64)
+        B = len(cu) - 1
+        scale = 1.0 / np.sqrt(D) if scale is None else scale
+        out = np.zeros((Tq, Hq, D), np.float64)
+        k_rot = is_rotated(self.fmt, False, self.flags)
+        v_rot = is_rotated(self.fmt, True, self.flags)
+
+        def run(job):
+            b, h = job
+            n, L = int(cu[b + 1] - cu[b]), int(seq_lens[b])
+            k, v = self.dequant(self.slots_of(block_table[b], L), h)
+            heads = slice(h * G, (h + 1) * G)
+            for i in range(n):
+                pos = L - n + i
+                if pos < 0:
+                    continue
+                row = int(cu[b]) + i
+                q = bf16_bits_to_f64(q_bf16[row, heads])
+                out[row, heads] = attend(q, k[:pos + 1], v[:pos + 1], k_rot, v_rot, scale)
+
+        jobs = [(b, h) for b in range(B) for h in range(self.H)
+                if cu[b + 1] > cu[b] and seq_lens[b] > 0]
+        if threads <= 1:
+            for j in jobs:
+                run(j)
+        else:
+            with ThreadPoolExecutor(threads) as ex:
+                list(ex.map(run, jobs))
+        return out
+
+
 def kv_elements(B: int, L: int, H_kv: int, S: int, d_head: int) -> int:
     """[llama.cpp] M_KV = 2 x B x L x H_kv x S x d_head (elements, K and V)."""
     return 2 * B * L * H_kv * S * d_head

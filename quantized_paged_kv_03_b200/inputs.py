@@ -237,6 +237,19 @@ def make_workload(cfg: int | ConfigSpec, fmt: str | None = None, seed: int | Non
     return Workload(spec, fmt, seed, B, H, Hq, D, P, seq_lens, bt, num_pages, k, v, q, starts)
 
 
+def prefill_queries(w: Workload, q_lens, seed: int | None = None):
+    """Query rows of a prefill chunk: q_lens[b] tokens of sequence b (its last
+    q_lens[b] tokens when q_lens[b] <= seq_lens[b]).  Returns (q, cu_q_lens):
+    bf16 bits [sum(q_lens), Hq, D], N(0, 1) like the decode queries, and the
+    int32 row offsets [B + 1] of each sequence's rows."""
+    q_lens = np.asarray(q_lens, np.int64)
+    cu = np.zeros(len(q_lens) + 1, np.int32)
+    cu[1:] = np.cumsum(q_lens)
+    r = _rng(w.seed if seed is None else seed, 6)
+    q = bf16_bits(r.standard_normal((int(cu[-1]), w.Hq, w.D), dtype=np.float32))
+    return q, cu
+
+
 def tensor_amax(x_bf16: np.ndarray) -> float:
     """Largest magnitude of a bf16 tensor (input statistic for a static scale)."""
     if x_bf16.size == 0:
