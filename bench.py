@@ -293,6 +293,111 @@ class Arm:
         return np.array(ts), h2d, d2h
 
 
+# ---------------------------------------------------------------- prefill arm
+
+def prefill_flops(seq_lens, q_lens, Hq: int, D: int) -> int:
+    """Algorithmic FLOPs of a chunked-prefill attention: 4 * D per (query row,
+    visible key) -- q.k and p.v, a multiply and an add per dimension each.
+    Query token i of a chunk of n sees L - n + i + 1 keys (causal)."""
+    keys = 0
+    for L, n in zip(seq_lens, q_lens):
+        first = int(L) - int(n) + 1
+        k = np.arange(first, first + int(n), dtype=np.int64)
+        keys += int(k[k > 0].sum())
+    return 4 * D * Hq * keys
+
+
+class PrefillArm:
+    """The chunked-prefill workload on the GPU: the prefix of every sequence in
+    the cache, the chunk's K/V rows, slots and queries resident in HBM.  One
+    step = append the chunk (kvq_append) + the causal attention of its queries
+    (kvq_prefill_attention)."""
+
+    def __init__(self, seed_offset: int = 0):
+        import torch
+        import quantized_paged_kv_03_b200 as K
+        self.torch = torch
+        spec, n = I.PREFILL, I.PREFILL_CHUNK
+        self.w = w = I.make_workload(spec, seed=I.PREFILL_SEED + 1000 * seed_offset)
+        fmt = spec.formats[0]
+        self.cache = K.KVCache(fmt, w.D, w.H, w.P, w.num_pages)
+        dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+        pre, pre_s, ch, ch_s = [], [], [], []
+        for b in range(w.B):
+            L, s0 = int(w.seq_lens[b]), int(w.starts[b])
+            pre.append(np.arange(s0, s0 + L - n))
+            pre_s.append(w.slots(b, 0, L - n))
+            ch.append(np.arange(s0 + L - n, s0 + L))
+            ch_s.append(w.slots(b, L - n, L))
+        pre, pre_s, ch = np.concatenate(pre), np.concatenate(pre_s), np.concatenate(ch)
+        step = 1 << 18
+        for i in range(0, len(pre), step):     # the prefix, untimed
+            r = pre[i:i + step]
+            self.cache.append(0, dev(w.k[r]).view(torch.bfloat16), dev(w.v[r]).view(torch.bfloat16),
+                              dev(pre_s[i:i + step]))
+        self.k_ch = dev(w.k[ch]).view(torch.bfloat16)
+        self.v_ch = dev(w.v[ch]).view(torch.bfloat16)
+        self.s_ch = dev(np.concatenate(ch_s))
+        self.q_lens = np.full(w.B, n, np.int64)
+        hq, cu = I.prefill_queries(w, self.q_lens)
+        self.q, self.cu = dev(hq).view(torch.bfloat16), dev(cu)
+        self.bt, self.sl = dev(w.block_table), dev(w.seq_lens)
+        self.out = torch.empty((int(cu[-1]), w.Hq, w.D), dtype=torch.float32, device="cuda")
+        self.max_q = n
+        self.chunk_tokens = int(len(ch))
+        self.flops = prefill_flops(w.seq_lens, self.q_lens, w.Hq, w.D)
+        self.tb = K.token_bytes(fmt, w.D)
+        self.kv_bytes = int(w.seq_lens.astype(np.int64).sum()) * w.H * self.tb
+        self.app_bytes = append_bytes(self.chunk_tokens, w, self.tb)
+        self.append_chunk()
+        torch.cuda.synchronize()
+        self.w.k = self.w.v = None
+
+    def append_chunk(self):
+        self.cache.append(0, self.k_ch, self.v_ch, self.s_ch)
+
+    def attend(self):
+        self.cache.prefill_attention(0, self.q, self.cu, self.bt, self.sl, self.max_q, out=self.out)
+
+    def step(self):
+        self.append_chunk()
+        self.attend()
+
+    run = Arm.run
+
+    def report(self, steps: int, warmup: int, flush, peak_tflops: float, peak_kind: str):
+        step_ms = float(self.run(steps, warmup, flush).mean())
+        att_ms = float(self.run(steps, warmup, flush, fn=self.attend).mean())
+        app_ms = float(self.run(steps, warmup, flush, fn=self.append_chunk).mean())
+        w = self.w
+        tflops = self.flops / (att_ms * 1e-3) / 1e12
+        return {
+            "workload": I.PREFILL.name,
+            "what": "append the chunk's K/V + causal attention of its queries over the cache "
+                    "(kvq_append + kvq_prefill_attention)",
+            "batch": w.B, "seq_len": int(w.seq_lens.max()), "chunk": self.max_q, "n_kv_heads": w.H,
+            "n_q_heads": w.Hq, "head_dim": w.D, "page_size": w.P, "format": I.PREFILL.formats[0],
+            "step_ms": round(step_ms, 5),
+            "chunk_tokens_per_s": round(self.chunk_tokens / (step_ms * 1e-3), 1),
+            "attention_ms": round(att_ms, 5), "attention_TFLOPs": round(tflops, 1),
+            "append_ms": round(app_ms, 5),
+            "append_GBps": round(self.app_bytes / (app_ms * 1e-3) / 1e9, 1),
+            "flops_per_launch": self.flops, "kv_bytes": self.kv_bytes,
+            "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": peak_tflops,
+                         "unit": "TFLOP/s", "frac": round(tflops / peak_tflops, 4), "traffic": None,
+                         "kernel": "prefill_kernel (mma.sync m16n8k16 fp16, fp32 accumulation)",
+                         "peak_source": f"{peak_kind} bf16_tflops (fp16 has the same dense rate)"},
+            "gpu_launches_per_step": 2,
+        }
+
+
+def load_tensor_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        return float(json.load(open(p))["bf16_tflops"]), "measured"
+    return 1590.0, "fallback"
+
+
 # ---------------------------------------------------------------- oracle arm
 
 def oracle_sample(cfg: int, fmt: str, budget_s: float = 12.0, threads: int | None = None):
@@ -410,6 +515,23 @@ def reference_arm(args):
     return 0
 
 
+def prefill_only(args):
+    """One JSON line with the prefill object alone (rank 0, one GPU)."""
+    import torch
+    from quantized_paged_kv_03_b200 import build
+    build.build()
+    flush = make_l2_flush(torch)
+    tpk, tkind = load_tensor_peak()
+    clocks_path = os.path.join(tempfile.gettempdir(), f"kvq_bench_clocks_{os.getpid()}_prefill.csv")
+    arm = PrefillArm()
+    clk = ClockSampler(clocks_path).__enter__()
+    rep = arm.report(args.steps, args.warmup, flush, tpk, tkind)
+    clk.__exit__(None, None, None)
+    rep["clocks"] = clk.summary(0)
+    print(json.dumps({"prefill": rep}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -422,11 +544,15 @@ def main():
                     help="workload index for the headline line (profiling a single kernel)")
     ap.add_argument("--format", default=None, help="format of that workload (default: its first)")
     ap.add_argument("--batch", type=int, default=None, help="fewer sequences (small profiling case)")
+    ap.add_argument("--prefill-only", action="store_true",
+                    help="time the chunked-prefill workload alone (profiling the prefill kernel)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         return reference_arm(args)
+    if args.prefill_only:
+        return prefill_only(args)
 
     import torch
     from quantized_paged_kv_03_b200 import build
@@ -491,6 +617,14 @@ def main():
                 del a
                 torch.cuda.empty_cache()
 
+    prefill = None
+    if not args.quick:
+        tpk, tkind = load_tensor_peak()
+        pa = PrefillArm(seed_offset=rank)
+        prefill = pa.report(args.steps, args.warmup, flush, tpk, tkind)
+        del pa
+        torch.cuda.empty_cache()
+
     clk.__exit__(None, None, None)
 
     cpu = None
@@ -532,6 +666,8 @@ def main():
             "wall_s_timed_region": round(t_wall, 3),
             "formats": formats,
         }
+        if prefill is not None:
+            line["prefill"] = prefill
         if cpu is not None:
             line["cpu_baseline"] = cpu
         print(json.dumps(line), flush=True)

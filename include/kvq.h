@@ -2,8 +2,9 @@
  * kvq.h -- C ABI of libkvq: a quantized paged KV cache for NVIDIA B200 (sm_100a).
  *
  * The library writes attention K/V rows into a paged cache in one of seven
- * storage formats and runs single-token (decode) GQA attention that reads the
- * pages back.  All compute runs in the library's own CUDA kernels; the caller
+ * storage formats and runs GQA attention that reads the pages back: for one
+ * new token per sequence (decode) and for a chunk of tokens (chunked
+ * prefill).  All compute runs in the library's own CUDA kernels; the caller
  * owns every byte of device memory (the library allocates nothing on the
  * device) and every CUDA stream.
  *
@@ -191,6 +192,36 @@ int kvq_decode_attention_noalloc(kvq_cache* cache, int32_t layer, const void* q,
                                  const int32_t* seq_lens, int32_t batch, int32_t max_seq_len,
                                  void* out, int32_t out_fp32, float softmax_scale, void* stream);
 
+/* Chunked-prefill attention: causal attention of a chunk of query tokens per
+ * sequence over the cache, the multi-token form of kvq_decode_attention for a
+ * prompt processed in chunks ([NInfer] K8V4 paragraph: the attention kernels
+ * over the quantized cache live under its "causal_cache" path).  The chunk's
+ * own K/V rows must already be appended (kvq_append).
+ *   q            bf16 [total_q][n_q_heads][head_dim]; the rows of sequence b are
+ *                cu_q_lens[b] .. cu_q_lens[b+1]-1: its n_b query tokens in order.
+ *   cu_q_lens    int32 [batch + 1], nondecreasing, cu_q_lens[0] = 0.
+ *   max_q_len    host: the largest n_b.  It sets the grid only: a longer chunk is
+ *                still computed in full, with less parallelism; 0 launches nothing.
+ *   block_table, max_pages_per_seq  as kvq_decode_attention.
+ *   seq_lens     int32 [batch]: cached tokens of each sequence, the chunk
+ *                included.  Query token i of sequence b sits at position
+ *                seq_lens[b] - n_b + i and attends positions [0, that position],
+ *                itself included; query head h reads kv-head
+ *                h / (n_q_heads / n_kv_heads).  A row whose position is negative
+ *                (n_b > seq_lens[b]) has no keys: its output row is zero.
+ *   out          [total_q][n_q_heads][head_dim], fp32 if out_fp32 else bf16.
+ *   softmax_scale  multiplier of q.k; 0 means 1/sqrt(head_dim).
+ * No workspace; the call allocates nothing.  Rotations as kvq_decode_attention.
+ * Arithmetic: q and the dequantised K/V enter the tensor cores as fp16 (bf16 for
+ * BF16 keys) with fp32 accumulation; dequantised values beyond fp16's range
+ * (|x| > 65504) saturate.  Page ids out of range, and pages past
+ * max_pages_per_seq, are replaced by page 0 and recorded in the device status
+ * word (bit 1); a pipeline wait that gives up sets bit 2. */
+int kvq_prefill_attention(kvq_cache* cache, int32_t layer, const void* q, int32_t n_q_heads,
+                          const int32_t* cu_q_lens, int32_t max_q_len, const int32_t* block_table,
+                          int32_t max_pages_per_seq, const int32_t* seq_lens, int32_t batch,
+                          void* out, int32_t out_fp32, float softmax_scale, void* stream);
+
 /* Test surface: stored values of the rows at `slots`, as fp32 code x scale in
  * the stored (rotated) domain.  k_out, v_out: fp32 [n][n_kv_heads][head_dim]. */
 int kvq_dequant(kvq_cache* cache, int32_t layer, const int64_t* slots, int32_t n,
@@ -210,7 +241,7 @@ int kvq_read_rows(kvq_cache* cache, int32_t layer, const int64_t* slots, int32_t
 int kvq_encode(int32_t code, const float* x, int64_t n, uint8_t* out, void* stream);
 
 /* Read (and optionally clear) the cache's device status word: bit 0 = a slot
- * out of range in kvq_append, bit 1 = a page id out of range in decode, bit 2 =
+ * out of range in kvq_append, bit 1 = a page id out of range in decode or prefill, bit 2 =
  * a decode pipeline wait gave up.  Synchronises `stream`. */
 int kvq_read_device_status(kvq_cache* cache, int32_t clear, uint32_t* status, void* stream);
 

@@ -1,5 +1,5 @@
-"""Python binding of libkvq: a quantized paged KV cache (append + decode
-attention) written for NVIDIA B200 (sm_100a).
+"""Python binding of libkvq: a quantized paged KV cache (append, decode
+attention and chunked-prefill attention) written for NVIDIA B200 (sm_100a).
 
 Argument marshalling only: every step of the path runs in the library's CUDA
 kernels (``csrc/``, C ABI in ``include/kvq.h``).  PyTorch supplies device
@@ -66,6 +66,8 @@ def lib() -> ctypes.CDLL:
                                              P, sz, P]),
         "kvq_decode_attention_noalloc": (ctypes.c_int, [P, i32, P, i32, P, i32, P, i32, i32, P, i32,
                                                         f32, P]),
+        "kvq_prefill_attention": (ctypes.c_int, [P, i32, P, i32, P, i32, P, i32, P, i32, P, i32, f32,
+                                                 P]),
         "kvq_dequant": (ctypes.c_int, [P, i32, P, i32, P, P, P]),
         "kvq_read_rows": (ctypes.c_int, [P, i32, P, i32, P, P, P, P, P]),
         "kvq_encode": (ctypes.c_int, [i32, P, i64, P, P]),
@@ -84,7 +86,8 @@ def lib() -> ctypes.CDLL:
 def exported_symbols():
     return ["kvq_token_bytes", "kvq_row_bytes", "kvq_cache_bytes", "kvq_cache_create",
             "kvq_cache_destroy", "kvq_append", "kvq_decode_workspace_bytes",
-            "kvq_decode_attention", "kvq_append_decode", "kvq_decode_attention_noalloc", "kvq_dequant", "kvq_read_rows", "kvq_encode",
+            "kvq_decode_attention", "kvq_append_decode", "kvq_decode_attention_noalloc",
+            "kvq_prefill_attention", "kvq_dequant", "kvq_read_rows", "kvq_encode",
             "kvq_read_device_status", "kvq_status_string", "kvq_version"]
 
 
@@ -290,6 +293,38 @@ class KVCache:
                                                   _ptr(out), int(out_fp32), float(softmax_scale),
                                                   _stream(stream)),
                "decode_attention_noalloc")
+        return out
+
+    def prefill_attention(self, layer: int, q, cu_q_lens, block_table, seq_lens, max_q_len: int | None = None,
+                          out=None, out_fp32: bool = True, softmax_scale: float = 0.0, stream=None):
+        """Causal attention of a chunk of query tokens per sequence (chunked
+        prefill).  q: bf16 [total_q, Hq, D], the rows of sequence b being
+        cu_q_lens[b] .. cu_q_lens[b+1]-1 (int32 [B+1]); seq_lens: int32 [B]
+        cached tokens, the chunk included (append its K/V first).  Query token
+        i of sequence b attends positions [0, seq_lens[b] - n_b + i].
+        max_q_len (the longest chunk) sizes the grid; None reads it from
+        cu_q_lens (a device-to-host copy)."""
+        import torch
+        _dev_tensor(q, torch.bfloat16, "q")
+        _dev_tensor(cu_q_lens, torch.int32, "cu_q_lens")
+        _dev_tensor(block_table, torch.int32, "block_table")
+        _dev_tensor(seq_lens, torch.int32, "seq_lens")
+        Tq, Hq, D = q.shape
+        B = seq_lens.numel()
+        if cu_q_lens.numel() != B + 1:
+            raise KVQError("prefill_attention: cu_q_lens must hold batch + 1 offsets")
+        if max_q_len is None:
+            max_q_len = int((cu_q_lens[1:] - cu_q_lens[:-1]).max().item()) if B else 0
+        if out is None:
+            out = torch.empty((Tq, Hq, D), dtype=torch.float32 if out_fp32 else torch.bfloat16,
+                              device=q.device)
+        else:
+            _dev_tensor(out, torch.float32 if out_fp32 else torch.bfloat16, "out")
+        _check(lib().kvq_prefill_attention(self._h, layer, _ptr(q), Hq, _ptr(cu_q_lens), int(max_q_len),
+                                           _ptr(block_table), block_table.shape[1], _ptr(seq_lens), B,
+                                           _ptr(out), int(out_fp32), float(softmax_scale),
+                                           _stream(stream)),
+               "prefill_attention")
         return out
 
     def dequant(self, layer: int, slots, stream=None):

@@ -14,7 +14,7 @@ CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libkvq.so")
 BUILD = os.path.join(HERE, "_build")
-SOURCES = ["kvq_api.cu", "kvq_append.cu", "kvq_decode.cu", "kvq_noalloc.cu"]
+SOURCES = ["kvq_api.cu", "kvq_append.cu", "kvq_decode.cu", "kvq_noalloc.cu", "kvq_prefill.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-O2",
          "--ftz=false", "--prec-div=true", "--prec-sqrt=true", "--fmad=true",

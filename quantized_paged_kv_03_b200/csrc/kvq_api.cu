@@ -7,6 +7,7 @@
 
 #include "../../include/kvq.h"
 #include "kvq_internal.h"
+#include "kvq_prefill.h"
 
 using namespace kvq;
 
@@ -223,6 +224,48 @@ static int decode_common(kvq_cache* cache, int32_t layer, const void* k_new, con
     p.k_scale = cache->tensor_scales[2 * layer];
     p.v_scale = cache->tensor_scales[2 * layer + 1];
     return cuda_status(launch_decode(p, plan, (cudaStream_t)stream));
+}
+
+int kvq_prefill_attention(kvq_cache* cache, int32_t layer, const void* q, int32_t n_q_heads,
+                          const int32_t* cu_q_lens, int32_t max_q_len, const int32_t* block_table,
+                          int32_t max_pages_per_seq, const int32_t* seq_lens, int32_t batch, void* out,
+                          int32_t out_fp32, float softmax_scale, void* stream) {
+    if (!cache || layer < 0 || layer >= cache->L.num_layers) return KVQ_ERR_ARG;
+    if (batch < 0 || n_q_heads < 1 || max_q_len < 0) return KVQ_ERR_ARG;
+    if (n_q_heads % cache->L.H) return KVQ_ERR_SHAPE;
+    if (!prefill_supported(cache->L.fmt, cache->L.D)) return KVQ_ERR_FORMAT;
+    if (batch == 0 || max_q_len == 0) return KVQ_OK;
+    if (!q || !cu_q_lens || !block_table || !seq_lens || !out || max_pages_per_seq < 1) return KVQ_ERR_ARG;
+    if (((uintptr_t)q & 15) || ((uintptr_t)out & 15)) return KVQ_ERR_ARG;
+    if (!(softmax_scale >= 0.f) || !isfinite(softmax_scale)) return KVQ_ERR_ARG;
+    PrefillPlan plan;
+    if (plan_prefill(cache->L, &plan) != cudaSuccess) return KVQ_ERR_SHAPE;
+    const int G = n_q_heads / cache->L.H;
+    const int64_t slots = ((int64_t)max_q_len * G + kPrefillRows - 1) / kPrefillRows;
+    const int64_t grid = (int64_t)batch * cache->L.H * slots;
+    if (grid > 0x7FFFFFFF) return KVQ_ERR_SHAPE;
+    PrefillParams p;
+    memset(&p, 0, sizeof(p));
+    p.L = cache->L;
+    p.slabs = layer_slabs(cache, layer);
+    p.q = (const uint16_t*)q;
+    p.cu_q_lens = cu_q_lens;
+    p.block_table = block_table;
+    p.max_pages = max_pages_per_seq;
+    p.seq_lens = seq_lens;
+    p.B = batch;
+    p.Hq = n_q_heads;
+    p.G = G;
+    p.slots = (int)slots;
+    p.out = out;
+    p.out_fp32 = out_fp32 ? 1 : 0;
+    const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)cache->L.D);
+    p.q_mult = scale * 1.4426950408889634f * cache->tensor_scales[2 * layer];
+    p.o_mult = cache->tensor_scales[2 * layer + 1];
+    p.rot_k = rot_of(cache, 0);
+    p.rot_v = rot_of(cache, 1);
+    p.status = (uint32_t*)cache->pool;
+    return cuda_status(launch_prefill(p, plan, grid, (cudaStream_t)stream));
 }
 
 int kvq_dequant(kvq_cache* cache, int32_t layer, const int64_t* slots, int32_t n, float* k_out, float* v_out,

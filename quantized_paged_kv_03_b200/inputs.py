@@ -71,6 +71,16 @@ CONFIGS = [
 
 SEED_BASE = 20261200
 
+# Chunked-prefill workload: the shape and value recipe of the INT8-G64 decode
+# workload above (8 kv-heads, 32 query heads, head_dim 256, 64-token pages, 2 %
+# of channels x20), with 4 sequences of 8192 cached tokens whose last
+# PREFILL_CHUNK tokens are the chunk being prefilled.
+PREFILL = ConfigSpec("int8_g64_prefill_b4_8k_chunk512", ("int8_g64",), B=4, n_kv_heads=8, n_q_heads=32,
+                     head_dim=256, page_size=64, lengths=("fixed", 8192),
+                     outlier_frac=0.02, outlier_gain=20.0)
+PREFILL_CHUNK = 512
+PREFILL_SEED = SEED_BASE + 500
+
 
 def bf16_bits(x: np.ndarray) -> np.ndarray:
     """fp32 -> bf16 bit patterns, round to nearest even (finite inputs)."""

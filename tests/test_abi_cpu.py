@@ -111,6 +111,15 @@ def test_calls_reject_bad_arguments_before_launch(L):
     assert L.kvq_decode_attention(h, 0, p, 4, p, 2, p, 2, 256, p, 1, 0.0, p, 1 << 20, None) == 3
     # batch 0 is a no-op
     assert L.kvq_decode_attention(h, 0, p, 4, p, 4, p, 0, 256, p, 1, 0.0, p, 1 << 20, None) == 0
+    # chunked prefill: layer out of range, heads not a multiple of kv-heads,
+    # negative scale, misaligned q; max_q_len 0 and batch 0 are no-ops
+    assert L.kvq_prefill_attention(h, 1, p, 4, p, 8, p, 4, p, 2, p, 1, 0.0, None) == 1
+    assert L.kvq_prefill_attention(h, 0, p, 5, p, 8, p, 4, p, 2, p, 1, 0.0, None) == 3
+    assert L.kvq_prefill_attention(h, 0, p, 4, p, 8, p, 4, p, 2, p, 1, -1.0, None) == 1
+    assert L.kvq_prefill_attention(h, 0, ctypes.c_void_p((1 << 21) + 8), 4, p, 8, p, 4, p, 2, p, 1, 0.0,
+                                   None) == 1
+    assert L.kvq_prefill_attention(h, 0, p, 4, p, 0, p, 4, p, 2, p, 1, 0.0, None) == 0
+    assert L.kvq_prefill_attention(h, 0, p, 4, p, 8, p, 4, p, 0, p, 1, 0.0, None) == 0
     assert L.kvq_encode(7, p, 4, p, None) == 1
     assert L.kvq_encode(0, p, 0, p, None) == 0
     assert L.kvq_read_rows(h, 0, p, 3, p, None, p, p, None) == 1     # K scales needed
