@@ -385,7 +385,7 @@ class PrefillArm:
             "flops_per_launch": self.flops, "kv_bytes": self.kv_bytes,
             "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": peak_tflops,
                          "unit": "TFLOP/s", "frac": round(tflops / peak_tflops, 4), "traffic": None,
-                         "kernel": "prefill_kernel (mma.sync m16n8k16 fp16, fp32 accumulation)",
+                         "kernel": "prefill_kernel (tcgen05.mma kind::f16, fp32 accumulation in tensor memory)",
                          "peak_source": f"{peak_kind} bf16_tflops (fp16 has the same dense rate)"},
             "gpu_launches_per_step": 2,
         }

@@ -14,19 +14,27 @@
 // Design (B200, sm_100a):
 //  * One CTA per (sequence, kv-head, block of 128 query rows); a row is a
 //    (query token, head of the GQA group) pair, so the G heads that share a
-//    kv-head share every key tile.  8 warps, 16 rows each, the whole head_dim
-//    per warp.  A (sequence, kv-head)'s heaviest block (its last rows, which
+//    kv-head share every key tile, and the 128 rows are the M of the tensor
+//    core's MMA.  A (sequence, kv-head)'s heaviest block (its last rows, which
 //    see the most keys) starts first.
 //  * Unlike decode, every key feeds many query rows: 4 x head_dim FLOPs per
 //    (row, key), a dense contraction for the tensor cores.  A key tile (64
-//    tokens, or fewer when the page size asks) arrives by cp.async.bulk into a
-//    two-stage ring; all threads then dequantise it once into fp16 tiles in
-//    shared memory, scales folded in (BF16 keys stay bf16, the format's own
-//    bits), and every warp reads its MMA operands from them with ldmatrix.
-//  * S = Q K^T and O += P V with mma.sync m16n8k16 and fp32 accumulators in
-//    registers; online softmax in the log2 domain; the causal mask is applied
-//    only on tiles that cross a warp's first position, and tiles past a warp's
-//    last position are skipped.
+//    tokens, or fewer when the page size or shared memory asks) arrives by
+//    cp.async.bulk into a two-stage ring; all 8 warps dequantise it once into
+//    fp16 operand tiles in shared memory (scales folded in; BF16 keys stay
+//    bf16, the format's own bits).
+//  * S = Q K^T and O += P V run on tcgen05.mma (M = 128, N = the tile or
+//    head_dim), issued by one thread, operands read from shared memory by the
+//    tensor core, accumulators in tensor memory (O in columns [0, D), S in
+//    [D, D + 64)).  Per tile: keys dequantised -> S issued -> values
+//    dequantised while S runs (after the previous P V has released them) ->
+//    every thread loads half of its row of S, the two halves exchange their
+//    maxima, P = 2^(s - m) goes to shared memory -> P V issued; the next
+//    tile's keys are dequantised while it runs.
+//  * Online softmax in the log2 domain with a lazy reference maximum: O in
+//    tensor memory is rescaled (load, multiply, store) only when a row's
+//    maximum grows by more than 2^8, so weights stay below 256.  The causal
+//    mask is applied on tiles that cross a lane group's first position.
 //  * Rotated K: q is rotated by the Hadamard-256 when staged (orthonormal, so
 //    q.k is unchanged); rotated V: each output row is rotated back in the
 //    epilogue (the matrix is symmetric and its own inverse).
@@ -39,12 +47,13 @@
 // values beyond fp16's range (|x| > 65504) saturate; the decode kernel, which
 // applies scales in fp32, has no such limit.
 #include "kvq_prefill.h"
+#include "kvq_tc.cuh"
 
 namespace kvq {
 namespace {
 
 constexpr long kPrefillWaitPolls = 1l << 22;
-constexpr int kMaxT = 64;   // largest key tile (tokens)
+constexpr int kMaxT = 64;   // largest key tile (tokens): S holds 64 tensor-memory columns
 
 // ------------------------------------------------------------ PTX helpers
 
@@ -82,32 +91,6 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
                  : "memory");
 }
 
-__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(addr));
-}
-
-template <bool BF16>
-__device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-    if constexpr (BF16) {
-        asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-            "{%0,%1,%2,%3};"
-            : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-    } else {
-        asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-            "{%0,%1,%2,%3};"
-            : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-    }
-}
-
 __device__ __forceinline__ uint32_t f16x2_of(float lo, float hi) {
     uint32_t r;
     asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
@@ -126,8 +109,8 @@ __device__ __forceinline__ uint32_t mul_f16x2(uint32_t a, uint32_t b) {
 __device__ __forceinline__ float2 f16x2_to_f32(uint32_t h) {
     return __half22float2(*reinterpret_cast<const __half2*>(&h));
 }
-// 2^x for x <= 0 (softmax weights); -inf gives 0.
-__device__ __forceinline__ float exp2_neg(float x) {
+// 2^x (softmax weights, x <= 8 here); -inf gives 0.
+__device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
@@ -136,22 +119,31 @@ __device__ __forceinline__ float exp2_neg(float x) {
 __device__ __forceinline__ uint32_t splat16(uint32_t h) { return (h & 0xFFFFu) * 0x10001u; }
 
 // ------------------------------------------------------------ tiles
+//
+// The operand tiles, 16-bit elements in 8 x 8 core matrices (kvq_tc.cuh):
+//  * q, 128 rows x D, the K-major A of S: core (r/8, d/8) at ((r/8)(D/8) + d/8) x 128
+//    (LBO 128, SBO 16 D);
+//  * keys and values, T rows x D: each 8-column block holds the T rows' 16-byte
+//    chunks in row order, core (t/8, d/8) at (d/8)(16 T) + (t/8) 128.  Keys are
+//    the K-major B of S (LBO 16 T along head_dim, SBO 128 along the tokens),
+//    values the MN-major B of P V (LBO 128 along the tokens, SBO 16 T along
+//    head_dim);
+//  * P, 128 rows x T, the K-major A of P V: core (r/8, t/8) at (t/8) 2048 + (r/8) 128
+//    (LBO 2048, SBO 128).
+// Rows of one 8-column block are consecutive 16-byte chunks, so threads that
+// write consecutive rows of a block write one contiguous run (no bank conflict).
 
-// Row stride (16-bit elements) of q and of the key/value tiles in shared
-// memory: 8 elements of padding put the 8 rows that one ldmatrix phase reads
-// in 8 distinct 16-byte bank groups.
-template <int D>
-constexpr int kTileStride = D + 8;
+__device__ __forceinline__ uint32_t kv_off(int t, int d, int T) { return (uint32_t)((d >> 3) * (T << 4) + (t << 4)); }
+__device__ __forceinline__ uint32_t p_off(int r, int c) { return (uint32_t)((c >> 3) * (kPrefillRows * 16) + (r << 4)); }
 
-// Dequantise one 16-byte code chunk (chunk j of a row, logical order) into
-// 16-bit elements at `d` (8, 16 or 32 of them, by the code width), with the
-// row's scales applied.
+// Dequantise one 16-byte code chunk (chunk j of row t, logical order) into the
+// tile, with the row's scales applied: 8, 16 or 32 elements by the code width.
 template <int KIND, int D>
-__device__ __forceinline__ void dequant_chunk(const uint4 w, const uint8_t* srow, int j, uint16_t* d) {
+__device__ __forceinline__ void dequant_chunk(const uint4 w, const uint8_t* srow, int j, uint8_t* tile, int t, int T) {
     constexpr int SB = kind_scale_bytes(KIND);
     const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
     if constexpr (kind_bits(KIND) == 16) {
-        *reinterpret_cast<uint4*>(d + j * 8) = w;           // bf16 keys / fp16 values: the stored bits
+        *reinterpret_cast<uint4*>(tile + kv_off(t, j * 8, T)) = w;   // bf16 keys / fp16 values: the stored bits
     } else if constexpr (kind_bits(KIND) == 4) {
         // 32 E2M1 codes (two groups of 16, UE4M3 scales): code x scale is exact in fp16
         const uint32_t sc = dec_e4m3x2_f16x2((uint32_t)srow[2 * j] | ((uint32_t)srow[2 * j + 1] << 8));
@@ -160,9 +152,10 @@ __device__ __forceinline__ void dequant_chunk(const uint4 w, const uint8_t* srow
 #pragma unroll
         for (int i = 0; i < 16; i++) h[i] = mul_f16x2(dec_e2m1x2_f16x2((ws[i >> 2] >> (8 * (i & 3))) & 0xFFu),
                                                       i < 8 ? s0 : s1);
-        uint4* o = reinterpret_cast<uint4*>(d + j * 32);
 #pragma unroll
-        for (int i = 0; i < 4; i++) o[i] = make_uint4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]);
+        for (int i = 0; i < 4; i++)
+            *reinterpret_cast<uint4*>(tile + kv_off(t, j * 32 + 8 * i, T)) =
+                make_uint4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]);
     } else {
         // 16 eight-bit codes, all in one scale group
         uint32_t h[8];
@@ -188,34 +181,34 @@ __device__ __forceinline__ void dequant_chunk(const uint4 w, const uint8_t* srow
                 h[i] = enc_f16x2_sat(f.x * sc, f.y * sc);
             }
         }
-        uint4* o = reinterpret_cast<uint4*>(d + j * 16);
-        o[0] = make_uint4(h[0], h[1], h[2], h[3]);
-        o[1] = make_uint4(h[4], h[5], h[6], h[7]);
+        *reinterpret_cast<uint4*>(tile + kv_off(t, j * 16, T)) = make_uint4(h[0], h[1], h[2], h[3]);
+        *reinterpret_cast<uint4*>(tile + kv_off(t, j * 16 + 8, T)) = make_uint4(h[4], h[5], h[6], h[7]);
     }
 }
 
 // Dequantise rows [0, T) of one array of a stage (codes: row stride
 // row_code_bytes, chunk-permuted as stored; scales: plain rows) into a tile.
-// Rows at or past `valid` lie beyond the sequence's last token and hold no
-// data: they are written as zeros, so that a masked key's weight 0 never meets
-// a non-finite value.
+// Thread c takes row t = c % T and chunk (c / T + t) % (chunks per row): the
+// 8 threads of a shared-memory phase read 8 different chunk columns and write
+// 8 consecutive rows.  Rows at or past `valid` lie beyond the sequence's last
+// token and hold no data: they are written as zeros, so that a masked key's
+// weight 0 never meets a non-finite value.
 template <int KIND, int D>
-__device__ __forceinline__ void dequant_tile(const uint8_t* codes, const uint8_t* scales, uint16_t* tile, int T,
+__device__ __forceinline__ void dequant_tile(const uint8_t* codes, const uint8_t* scales, uint8_t* tile, int T,
                                              int valid, int tid) {
     constexpr int CB = row_code_bytes(KIND, D), SB = row_scale_bytes(KIND, D);
     constexpr int CPR = CB / 16;                       // chunks per row (a power of two)
     constexpr int EPC = 128 / kind_bits(KIND);         // elements per chunk
     for (int c = tid; c < T * CPR; c += kPrefillThreads) {
-        const int t = c / CPR, j = c % CPR;
-        uint16_t* d = tile + t * kTileStride<D>;
+        const int t = c % T, j = (c / T + t) & (CPR - 1);
         if (t >= valid) {
-            uint4* o = reinterpret_cast<uint4*>(d + j * EPC);
 #pragma unroll
-            for (int i = 0; i < EPC / 8; i++) o[i] = make_uint4(0, 0, 0, 0);
+            for (int i = 0; i < EPC / 8; i++)
+                *reinterpret_cast<uint4*>(tile + kv_off(t, j * EPC + 8 * i, T)) = make_uint4(0, 0, 0, 0);
             continue;
         }
         const uint4 w = *reinterpret_cast<const uint4*>(codes + t * CB + ((j ^ row_swizzle(KIND, D, t)) << 4));
-        dequant_chunk<KIND, D>(w, scales + t * SB, j, d);
+        dequant_chunk<KIND, D>(w, scales + t * SB, j, tile, t, T);
     }
 }
 
@@ -224,7 +217,7 @@ __device__ __forceinline__ void dequant_tile(const uint8_t* codes, const uint8_t
 // (rotated by the Hadamard-256 first when K is rotated), or the bf16 bits
 // themselves for BF16 keys; rows past the chunk are zeros.  One warp per row.
 template <int D, bool QBF16>
-__device__ __forceinline__ void stage_q(const PrefillParams& p, uint16_t* sQ, int64_t qrow0, int hh, int64_t R0,
+__device__ __forceinline__ void stage_q(const PrefillParams& p, uint8_t* sQ, int64_t qrow0, int hh, int64_t R0,
                                         int64_t rows_total, int warp, int lane) {
     constexpr int EPL = D / 32;
     for (int r = warp; r < kPrefillRows; r += kPrefillThreads / 32) {
@@ -260,11 +253,10 @@ __device__ __forceinline__ void stage_q(const PrefillParams& p, uint16_t* sQ, in
 #pragma unroll
             for (int i = 0; i < EPL / 2; i++) h[i] = enc_f16x2_sat(x[2 * i], x[2 * i + 1]);
         }
-        uint16_t* d = sQ + r * kTileStride<D> + lane * EPL;
         if constexpr (EPL == 8) {
-            *reinterpret_cast<uint4*>(d) = make_uint4(h[0], h[1], h[2], h[3]);
+            *reinterpret_cast<uint4*>(sQ + tc::blk(r, lane * 8, D)) = make_uint4(h[0], h[1], h[2], h[3]);
         } else {
-            *reinterpret_cast<uint2*>(d) = make_uint2(h[0], h[1]);
+            *reinterpret_cast<uint2*>(sQ + tc::blk(r, (lane * 4) & ~7, D) + (lane & 1) * 8) = make_uint2(h[0], h[1]);
         }
     }
 }
@@ -273,21 +265,22 @@ __device__ __forceinline__ void stage_q(const PrefillParams& p, uint16_t* sQ, in
 
 template <int KK, int KV, int D>
 __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const PrefillParams p) {
-    constexpr bool KBF = (KK == RK_BF16RAW);   // bf16 keys: S on the bf16 MMA
-    constexpr int TS = kTileStride<D>;
-    constexpr int NO = D / 8;                  // output n-tiles (8 dims each)
-    constexpr int NS = kMaxT / 8;              // score n-tiles of the largest key tile
+    constexpr bool KBF = (KK == RK_BF16RAW);   // bf16 keys: S on bf16 operands
     constexpr int EPL = D / 32;                // output values per lane in the epilogue
     constexpr int OST = D + 4;                 // fp32 row stride of the output staging
-    extern __shared__ __align__(128) uint8_t smem[];
-    const int T = p.T, nts = T / 8;
-    uint16_t* sQ = reinterpret_cast<uint16_t*>(smem);
-    uint16_t* sK = sQ + kPrefillRows * TS;
-    uint16_t* sV = sK + T * TS;
+    constexpr uint32_t kCols = D == 256 ? 512 : 256;   // tensor memory: O in [0, D), S in [D, D + 64)
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const int T = p.T;
+    uint8_t* sQ = smem;
+    uint8_t* sK = sQ + kPrefillRows * D * 2;
+    uint8_t* sV = sK + T * D * 2;
+    uint8_t* sP = sV + T * D * 2;
     float* sO = reinterpret_cast<float*>(smem);
     uint8_t* ring = smem + prefill_region0(D, T);
     uint64_t* bars = reinterpret_cast<uint64_t*>(ring + (size_t)p.stages * p.st_bytes);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + p.stages);
+    float* red = reinterpret_cast<float*>(bars + p.stages + 2);   // [2][128]: per-half row values
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(red + 2 * kPrefillRows);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     int64_t idx = blockIdx.x;
@@ -302,12 +295,25 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const Prefi
     const int64_t nblk = (rows_total + kPrefillRows - 1) / kPrefillRows;
     if (slot >= nblk) return;
 
+    const uint32_t barS = smem_addr(&bars[p.stages]), barO = smem_addr(&bars[p.stages + 1]);
     if (tid == 0) {
-        for (int s = 0; s < p.stages; s++) mbar_init(smem_addr(&bars[s]), 1);
+        for (int s = 0; s < p.stages + 2; s++) mbar_init(smem_addr(&bars[s]), 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
+    if (warp == 0) tc::alloc(smem_addr(tslot), kCols);
+    tc::fence_before();
     __syncthreads();
+    tc::fence_after();
+    const uint32_t tmem = *tslot;
+    const uint32_t tO = tmem, tS = tmem + D;
+
+    // this thread's TMEM lane (= row of the block) and column half
+    const int g4 = warp & 3, h = warp >> 2;
+    const int r = g4 * 32 + lane;
+    const uint32_t lane_bits = (uint32_t)(g4 * 32) << 16;
+    const uint32_t idS = tc::idesc_f16(KBF, false, T), idO = tc::idesc_f16(false, true, D);
+    const uint32_t aQ = smem_addr(sQ), aK = smem_addr(sK), aV = smem_addr(sV), aP = smem_addr(sP);
 
     // key tile k of this sequence into stage s: the whole page slab in one copy
     // when the tile is the page, else the tile's rows of the slab's four arrays
@@ -337,14 +343,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const Prefi
             if (nvs) bulk_g2s(dst + (uint32_t)p.st_vs, src + p.L.off_vs + r0 * p.L.vs, nvs, bar);
         }
     };
+    auto wait_or_flag = [&](uint32_t bar, uint32_t phase) {
+        if (!mbar_wait(bar, phase, abort_flag) && lane == 0) atomicOr(p.status, kStatusWaitTimeout);
+    };
 
-    // ldmatrix lane addresses: q rows (A operand), key rows (B of S), value
-    // rows (B of O, transposed on load)
-    const uint32_t qa_addr = smem_addr(sQ + (warp * 16 + (lane & 15)) * TS + (lane >> 4) * 8);
-    const uint32_t kb_addr = smem_addr(sK + (lane & 7) * TS + (lane >> 3) * 8);
-    const uint32_t vb_addr = smem_addr(sV + ((lane & 7) + ((lane >> 3) & 1) * 8) * TS + (lane >> 4) * 8);
-
-    uint32_t seq = 0;   // key tiles consumed by this CTA: stage = seq % stages, phase = seq / stages
+    uint32_t seq = 0;   // key tiles consumed by this CTA: ring stage seq % stages, phase seq / stages
+    uint32_t rnd = 0;   // MMA rounds (one S and one O per tile): phase of barS and barO
     for (int64_t jb = slot; jb < nblk; jb += p.slots) {
         const int64_t R0 = (nblk - 1 - jb) * kPrefillRows;   // the heaviest block first
         const int64_t r_last = min(R0 + kPrefillRows, rows_total) - 1;
@@ -353,176 +357,182 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const Prefi
         if (tid == 0)
             for (int k = 0; k < p.stages && k < ntiles; k++) issue(seq + k, k);
         stage_q<D, KBF>(p, sQ, qrow0, hh, R0, rows_total, warp, lane);
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 
-        // this thread's two rows (lane/4 and lane/4 + 8 of the warp's 16) and the
-        // warp's position range; rows past the chunk get position -1 (no keys)
-        const int64_t ra = R0 + warp * 16 + (lane >> 2), rb = ra + 8;
-        const int pos_a = ra < rows_total ? Ls - n + (int)(ra / p.G) : -1;
-        const int pos_b = rb < rows_total ? Ls - n + (int)(rb / p.G) : -1;
-        const int64_t w0 = R0 + warp * 16;
-        const int wpos_min = w0 + 15 < rows_total ? Ls - n + (int)(w0 / p.G) : -1;
-        const int wpos_max = w0 < rows_total ? Ls - n + (int)((min(w0 + 15, rows_total - 1)) / p.G) : -1;
-
-        float O[NO][4];
-#pragma unroll
-        for (int i = 0; i < NO; i++) O[i][0] = O[i][1] = O[i][2] = O[i][3] = 0.f;
-        float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
+        // this thread's row position (-1: past the chunk, no keys) and the
+        // smallest position among the 32 rows of its lane group
+        const int64_t gr = R0 + r;
+        const int pos = gr < rows_total ? Ls - n + (int)(gr / p.G) : -1;
+        const int64_t gfirst = R0 + g4 * 32;
+        const int gpos_min = gfirst + 31 < rows_total ? Ls - n + (int)(gfirst / p.G) : -1;
+        float m_ref = -INFINITY, l_part = 0.f;
         __syncthreads();   // q staged
 
-        for (int k = 0; k < ntiles; k++, seq++) {
+        for (int k = 0; k < ntiles; k++, seq++, rnd++) {
             const int s = (int)(seq % (uint32_t)p.stages);
             const uint8_t* st = ring + (size_t)s * p.st_bytes;
-            if (!mbar_wait(smem_addr(&bars[s]), (seq / (uint32_t)p.stages) & 1u, abort_flag) && lane == 0)
-                atomicOr(p.status, kStatusWaitTimeout);
+            wait_or_flag(smem_addr(&bars[s]), (seq / (uint32_t)p.stages) & 1u);
             const int t0 = k * T;
             const int valid = min(T, Ls - t0);
+            // keys first: S of this tile can start while the values are dequantised
             dequant_tile<KK, D>(st, st + p.st_ks, sK, T, valid, tid);
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncthreads();
+            if (tid == 0) {
+                tc::fence_after();
+#pragma unroll
+                for (int kk = 0; kk < D / 16; kk++)
+                    tc::mma_f16(tS, tc::sdesc(aQ + 256 * kk, 128, 16 * D), tc::sdesc(aK + kk * 32 * T, 16 * T, 128),
+                                idS, kk > 0);
+                tc::commit(barS);
+            }
+            if (k > 0) {   // the previous P V still reads the value and P tiles
+                wait_or_flag(barO, (rnd - 1) & 1u);
+                tc::fence_after();
+            }
             dequant_tile<KV, D>(st + p.st_vc, st + p.st_vs, sV, T, valid, tid);
-            __syncthreads();   // tiles ready; the stage is free again
-            if (tid == 0 && k + p.stages < ntiles) issue(seq + p.stages, k + p.stages);
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 
-            if (t0 <= wpos_max) {
-                // ---- S = Q K^T: 16 rows x T keys, head_dim in steps of 32
-                float S[NS][4];
+            // ---- scores of this thread's row, columns [32 h, 32 h + 32) of the tile
+            wait_or_flag(barS, rnd & 1u);
+            tc::fence_after();
+            const int c0 = h * 32;
+            const bool active = c0 < T;   // with tiles of 32 or 16 keys the second half has none
+            float sv[32];
+            float mx = -INFINITY;
+            if (active) {
+                uint32_t v[32];
+                tc::ld32(tS + lane_bits + c0, v);
+                tc::wait_ld();
+                const bool mask = t0 + T - 1 > gpos_min;
 #pragma unroll
-                for (int i = 0; i < NS; i++) S[i][0] = S[i][1] = S[i][2] = S[i][3] = 0.f;
-#pragma unroll
-                for (int kp = 0; kp < D / 32; kp++) {
-                    uint32_t qa0[4], qa1[4];
-                    ldsm_x4(qa0, qa_addr + kp * 64);
-                    ldsm_x4(qa1, qa_addr + kp * 64 + 32);
-#pragma unroll
-                    for (int nt = 0; nt < NS; nt++) {
-                        if (nt < nts) {
-                            uint32_t kb[4];
-                            ldsm_x4(kb, kb_addr + nt * 8 * TS * 2 + kp * 64);
-                            mma16816<KBF>(S[nt], qa0, kb[0], kb[1]);
-                            mma16816<KBF>(S[nt], qa1, kb[2], kb[3]);
-                        }
-                    }
-                }
-                // ---- online softmax (log2 domain), causal mask where the tile
-                // crosses a row's position
-                const bool mask = t0 + T - 1 > wpos_min;
-                float mx_a = -INFINITY, mx_b = -INFINITY;
-#pragma unroll
-                for (int nt = 0; nt < NS; nt++) {
-                    if (nt < nts) {
-                        const int key = t0 + nt * 8 + (lane & 3) * 2;
-                        float s0 = S[nt][0] * p.q_mult, s1 = S[nt][1] * p.q_mult;
-                        float s2 = S[nt][2] * p.q_mult, s3 = S[nt][3] * p.q_mult;
-                        if (mask) {
-                            if (key > pos_a) s0 = -INFINITY;
-                            if (key + 1 > pos_a) s1 = -INFINITY;
-                            if (key > pos_b) s2 = -INFINITY;
-                            if (key + 1 > pos_b) s3 = -INFINITY;
-                        }
-                        S[nt][0] = s0; S[nt][1] = s1; S[nt][2] = s2; S[nt][3] = s3;
-                        mx_a = fmaxf(mx_a, fmaxf(s0, s1));
-                        mx_b = fmaxf(mx_b, fmaxf(s2, s3));
-                    }
-                }
-                mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 1));
-                mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 2));
-                mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 1));
-                mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 2));
-                const float mn_a = fmaxf(m_a, mx_a), mn_b = fmaxf(m_b, mx_b);
-                const float base_a = mn_a == -INFINITY ? 0.f : mn_a;
-                const float base_b = mn_b == -INFINITY ? 0.f : mn_b;
-                const float corr_a = exp2_neg(m_a - base_a), corr_b = exp2_neg(m_b - base_b);
-                m_a = mn_a;
-                m_b = mn_b;
-                float rs_a = 0.f, rs_b = 0.f;
-                uint32_t pa[NS / 2][4];
-#pragma unroll
-                for (int kt = 0; kt < NS / 2; kt++) {
-                    if (2 * kt < nts) {
-                        const float p00 = exp2_neg(S[2 * kt][0] - base_a), p01 = exp2_neg(S[2 * kt][1] - base_a);
-                        const float p02 = exp2_neg(S[2 * kt][2] - base_b), p03 = exp2_neg(S[2 * kt][3] - base_b);
-                        const float p10 = exp2_neg(S[2 * kt + 1][0] - base_a), p11 = exp2_neg(S[2 * kt + 1][1] - base_a);
-                        const float p12 = exp2_neg(S[2 * kt + 1][2] - base_b), p13 = exp2_neg(S[2 * kt + 1][3] - base_b);
-                        rs_a += (p00 + p01) + (p10 + p11);
-                        rs_b += (p02 + p03) + (p12 + p13);
-                        pa[kt][0] = f16x2_of(p00, p01);
-                        pa[kt][1] = f16x2_of(p02, p03);
-                        pa[kt][2] = f16x2_of(p10, p11);
-                        pa[kt][3] = f16x2_of(p12, p13);
-                    }
-                }
-                l_a = l_a * corr_a + rs_a;
-                l_b = l_b * corr_b + rs_b;
-                if (__any_sync(0xffffffffu, corr_a != 1.f || corr_b != 1.f)) {
-#pragma unroll
-                    for (int i = 0; i < NO; i++) {
-                        O[i][0] *= corr_a; O[i][1] *= corr_a;
-                        O[i][2] *= corr_b; O[i][3] *= corr_b;
-                    }
-                }
-                // ---- O += P V: 16 keys per k-step, 16 output dims per load
-#pragma unroll
-                for (int kt = 0; kt < NS / 2; kt++) {
-                    if (2 * kt < nts) {
-#pragma unroll
-                        for (int dp = 0; dp < D / 16; dp++) {
-                            uint32_t vb[4];
-                            ldsm_x4_t(vb, vb_addr + (kt * 16 * TS + dp * 16) * 2);
-                            mma16816<false>(O[2 * dp], pa[kt], vb[0], vb[1]);
-                            mma16816<false>(O[2 * dp + 1], pa[kt], vb[2], vb[3]);
-                        }
-                    }
+                for (int i = 0; i < 32; i++) {
+                    float x = __uint_as_float(v[i]) * p.q_mult;
+                    if (c0 + i >= T || (mask && t0 + c0 + i > pos)) x = -INFINITY;
+                    sv[i] = x;
+                    mx = fmaxf(mx, x);
                 }
             }
-            __syncthreads();   // tiles consumed
+            red[h * kPrefillRows + r] = mx;
+            tc::fence_before();
+            __syncthreads();   // row maxima exchanged; the stage and the S columns are free
+            if (tid == 0 && k + p.stages < ntiles) issue(seq + p.stages, k + p.stages);
+            // lazy rescale: keep the reference max unless the tile's max exceeds it by
+            // more than 2^8 (weights up to 256 are safe in fp16 and fp32)
+            const float mt = fmaxf(red[r], red[kPrefillRows + r]);
+            float corr = 1.f;
+            const bool resc = mt > m_ref + 8.f;
+            if (resc) {
+                corr = ex2(m_ref - mt);
+                m_ref = mt;
+            }
+            const float base = m_ref == -INFINITY ? 0.f : m_ref;
+            float rs = 0.f;
+            if (active) {
+#pragma unroll
+                for (int q8 = 0; q8 < 4; q8++) {
+                    uint32_t hw[4];
+#pragma unroll
+                    for (int i = 0; i < 4; i++) {
+                        const float pa = ex2(sv[8 * q8 + 2 * i] - base), pb = ex2(sv[8 * q8 + 2 * i + 1] - base);
+                        rs += pa + pb;
+                        hw[i] = f16x2_of(pa, pb);
+                    }
+                    if (c0 + 8 * q8 < T)
+                        *reinterpret_cast<uint4*>(sP + p_off(r, c0 + 8 * q8)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                }
+            }
+            l_part = l_part * corr + rs;
+            if (k > 0 && __any_sync(0xffffffffu, resc)) {
+                // O of this thread's row, columns [h D/2, h D/2 + D/2), times corr
+#pragma unroll 1
+                for (int cc = 0; cc < D / 2; cc += 32) {
+                    uint32_t v[32];
+                    const uint32_t ta = tO + lane_bits + h * (D / 2) + cc;
+                    tc::ld32(ta, v);
+                    tc::wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; i++) v[i] = __float_as_uint(__uint_as_float(v[i]) * corr);
+                    tc::st32(ta, v);
+                }
+                tc::wait_st();
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            tc::fence_before();
+            __syncthreads();   // P and the value tile written, O rescaled
+            if (tid == 0) {
+                tc::fence_after();
+#pragma unroll
+                for (int kk = 0; kk < kMaxT / 16; kk++)
+                    if (kk < T / 16)
+                        tc::mma_f16(tO, tc::sdesc(aP + kk * 2 * (kPrefillRows * 16), kPrefillRows * 16, 128),
+                                    tc::sdesc(aV + 256 * kk, 128, 16 * T), idO, k > 0 || kk > 0);
+                tc::commit(barO);
+            }
         }
 
-        // ---- epilogue: normalise, stage the warp's rows, rotate V back, store
-        l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
-        l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
-        l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
-        l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
-        const float inv_a = l_a > 0.f ? p.o_mult / l_a : 0.f;
-        const float inv_b = l_b > 0.f ? p.o_mult / l_b : 0.f;
-        float* so = sO + warp * 16 * OST;
-#pragma unroll
-        for (int i = 0; i < NO; i++) {
-            const int col = i * 8 + (lane & 3) * 2;
-            *reinterpret_cast<float2*>(so + (lane >> 2) * OST + col) = make_float2(O[i][0] * inv_a, O[i][1] * inv_a);
-            *reinterpret_cast<float2*>(so + ((lane >> 2) + 8) * OST + col) =
-                make_float2(O[i][2] * inv_b, O[i][3] * inv_b);
+        // ---- epilogue: normalise, stage the rows, rotate V back, store
+        if (ntiles > 0) {
+            wait_or_flag(barO, (rnd - 1) & 1u);
+            tc::fence_after();
         }
-        __syncwarp();
-        for (int r = 0; r < 16; r++) {
-            const int64_t gr = w0 + r;
-            if (gr >= rows_total) break;
+        red[h * kPrefillRows + r] = l_part;
+        __syncthreads();
+        const float l = red[r] + red[kPrefillRows + r];
+        const float inv = l > 0.f ? p.o_mult / l : 0.f;
+        float* so = sO + r * OST + h * (D / 2);
+#pragma unroll 1
+        for (int cc = 0; cc < D / 2; cc += 32) {
+            uint32_t v[32];
+            if (ntiles > 0) {
+                tc::ld32(tO + lane_bits + h * (D / 2) + cc, v);
+                tc::wait_ld();
+            }
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+                *reinterpret_cast<float4*>(so + cc + i) =
+                    ntiles > 0 ? make_float4(__uint_as_float(v[i]) * inv, __uint_as_float(v[i + 1]) * inv,
+                                             __uint_as_float(v[i + 2]) * inv, __uint_as_float(v[i + 3]) * inv)
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        tc::fence_before();
+        __syncthreads();   // output rows staged; tensor memory reads done
+        for (int rr = warp; rr < kPrefillRows; rr += kPrefillThreads / 32) {
+            const int64_t grr = R0 + rr;
+            if (grr >= rows_total) break;
             float x[EPL];
 #pragma unroll
             for (int i = 0; i < EPL; i += 4) {
-                const float4 v = *reinterpret_cast<const float4*>(so + r * OST + lane * EPL + i);
+                const float4 v = *reinterpret_cast<const float4*>(sO + rr * OST + lane * EPL + i);
                 x[i] = v.x; x[i + 1] = v.y; x[i + 2] = v.z; x[i + 3] = v.w;
             }
             if constexpr (D == 256) {
                 if (p.rot_v) fwht256_warp(x, lane);
             }
-            const int64_t i_tok = gr / p.G, g = gr % p.G;
+            const int64_t i_tok = grr / p.G, g = grr % p.G;
             const int64_t o = ((qrow0 + i_tok) * p.Hq + (int64_t)hh * p.G + g) * D + lane * EPL;
             if (p.out_fp32) {
                 float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + o);
 #pragma unroll
                 for (int i = 0; i < EPL / 4; i++) dst[i] = make_float4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
             } else {
-                uint32_t h[EPL / 2];
+                uint32_t hb[EPL / 2];
 #pragma unroll
-                for (int i = 0; i < EPL / 2; i++) h[i] = bf16x2_of(x[2 * i], x[2 * i + 1]);
+                for (int i = 0; i < EPL / 2; i++) hb[i] = bf16x2_of(x[2 * i], x[2 * i + 1]);
                 uint16_t* dst = static_cast<uint16_t*>(p.out) + o;
                 if constexpr (EPL == 8) {
-                    *reinterpret_cast<uint4*>(dst) = make_uint4(h[0], h[1], h[2], h[3]);
+                    *reinterpret_cast<uint4*>(dst) = make_uint4(hb[0], hb[1], hb[2], hb[3]);
                 } else {
-                    *reinterpret_cast<uint2*>(dst) = make_uint2(h[0], h[1]);
+                    *reinterpret_cast<uint2*>(dst) = make_uint2(hb[0], hb[1]);
                 }
             }
         }
         __syncthreads();   // the shared region is free for the next block
     }
+    tc::fence_before();
+    __syncthreads();
+    tc::fence_after();
+    if (warp == 0) tc::dealloc(tmem, kCols);
 }
 
 }  // namespace
@@ -548,7 +558,7 @@ cudaError_t plan_prefill(const Layout& L, PrefillPlan* plan) {
         q.st_vc = q.st_ks + (int)align16((int64_t)T * L.ks);
         q.st_vs = q.st_vc + (int)align16((int64_t)T * L.vc);
         q.st_bytes = q.st_vs + (int)align16((int64_t)T * L.vs);
-        q.smem = (size_t)prefill_region0(L.D, T) + (size_t)stages * q.st_bytes + 8 * stages + 16;
+        q.smem = (size_t)prefill_region0(L.D, T) + (size_t)stages * q.st_bytes + (size_t)prefill_tail_bytes(stages);
         if (q.smem <= kSmemLimit) {
             *plan = q;
             return cudaSuccess;

@@ -10,14 +10,18 @@ constexpr int kPrefillRows = 128;    // query rows (token, head) per CTA: 8 warp
 constexpr int kPrefillThreads = 256;
 
 // Bytes of the first shared-memory region of a CTA at head_dim D and key tile
-// T: q (128 rows) and the key and value tiles (T rows each) during the key
-// loop, 16-bit elements with rows padded by 8; the per-warp fp32 output rows
-// (padded by 4) in the epilogue.  Rounded up to 128 bytes.
+// T: during the key loop the 16-bit operand tiles of the tensor core -- q
+// (128 x D), keys and values (T x D each) and the probabilities P (128 x T);
+// in the epilogue the fp32 output rows (128 x (D + 4)).  Rounded up to 1 KB.
 KVQ_HD constexpr int64_t prefill_region0(int D, int T) {
-    const int64_t qkv = (int64_t)(kPrefillRows + 2 * T) * (D + 8) * 2;
-    const int64_t osm = (int64_t)(kPrefillThreads / 32) * 16 * (D + 4) * 4;
-    return ((qkv > osm ? qkv : osm) + 127) & ~int64_t(127);
+    const int64_t ops = ((int64_t)kPrefillRows * D + 2 * (int64_t)T * D + (int64_t)kPrefillRows * T) * 2;
+    const int64_t osm = (int64_t)kPrefillRows * (D + 4) * 4;
+    return ((ops > osm ? ops : osm) + 1023) & ~int64_t(1023);
 }
+// Bytes after the stage ring: the ring's mbarriers, the S and O completion
+// mbarriers, the row exchange buffer (2 x 128 floats), the tensor-memory
+// address and the abort flag.
+KVQ_HD constexpr int64_t prefill_tail_bytes(int stages) { return 8 * (stages + 2) + 2 * kPrefillRows * 4 + 16; }
 
 struct PrefillParams {
     Layout L;
