@@ -190,25 +190,39 @@ __device__ __forceinline__ void dequant_chunk(const uint4 w, const uint8_t* srow
 // row_code_bytes, chunk-permuted as stored; scales: plain rows) into a tile.
 // Thread c takes row t = c % T and chunk (c / T + t) % (chunks per row): the
 // 8 threads of a shared-memory phase read 8 different chunk columns and write
-// 8 consecutive rows.  Rows at or past `valid` lie beyond the sequence's last
-// token and hold no data: they are written as zeros, so that a masked key's
-// weight 0 never meets a non-finite value.
+// 8 consecutive rows.  A thread loads all its chunks before converting any, so
+// their shared-memory latencies overlap.  Rows at or past `valid` lie beyond
+// the sequence's last token and hold no data: they are written as zeros, so
+// that a masked key's weight 0 never meets a non-finite value.
 template <int KIND, int D>
 __device__ __forceinline__ void dequant_tile(const uint8_t* codes, const uint8_t* scales, uint8_t* tile, int T,
-                                             int valid, int tid) {
+                                             int lgT, int valid, int tid) {
     constexpr int CB = row_code_bytes(KIND, D), SB = row_scale_bytes(KIND, D);
     constexpr int CPR = CB / 16;                       // chunks per row (a power of two)
     constexpr int EPC = 128 / kind_bits(KIND);         // elements per chunk
-    for (int c = tid; c < T * CPR; c += kPrefillThreads) {
-        const int t = c % T, j = (c / T + t) & (CPR - 1);
+    constexpr int NPT = (kMaxT * CPR + kPrefillThreads - 1) / kPrefillThreads;   // chunks per thread, at most
+    const int total = T * CPR;
+    uint4 w[NPT];
+#pragma unroll
+    for (int i = 0; i < NPT; i++) {
+        const int c = tid + i * kPrefillThreads;
+        const int t = c & (T - 1), j = ((c >> lgT) + t) & (CPR - 1);
+        w[i] = make_uint4(0, 0, 0, 0);
+        if (c < total && t < valid)
+            w[i] = *reinterpret_cast<const uint4*>(codes + t * CB + ((j ^ row_swizzle(KIND, D, t)) << 4));
+    }
+#pragma unroll
+    for (int i = 0; i < NPT; i++) {
+        const int c = tid + i * kPrefillThreads;
+        const int t = c & (T - 1), j = ((c >> lgT) + t) & (CPR - 1);
+        if (c >= total) continue;
         if (t >= valid) {
 #pragma unroll
-            for (int i = 0; i < EPC / 8; i++)
-                *reinterpret_cast<uint4*>(tile + kv_off(t, j * EPC + 8 * i, T)) = make_uint4(0, 0, 0, 0);
-            continue;
+            for (int e = 0; e < EPC / 8; e++)
+                *reinterpret_cast<uint4*>(tile + kv_off(t, j * EPC + 8 * e, T)) = make_uint4(0, 0, 0, 0);
+        } else {
+            dequant_chunk<KIND, D>(w[i], scales + t * SB, j, tile, t, T);
         }
-        const uint4 w = *reinterpret_cast<const uint4*>(codes + t * CB + ((j ^ row_swizzle(KIND, D, t)) << 4));
-        dequant_chunk<KIND, D>(w, scales + t * SB, j, tile, t, T);
     }
 }
 
@@ -270,7 +284,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const Prefi
     constexpr int OST = D + 4;                 // fp32 row stride of the output staging
     constexpr uint32_t kCols = D == 256 ? 512 : 256;   // tensor memory: O in [0, D), S in [D, D + 64)
     extern __shared__ __align__(1024) uint8_t smem[];
-    const int T = p.T;
+    const int T = p.T, lgT = 31 - __clz(T);
     uint8_t* sQ = smem;
     uint8_t* sK = sQ + kPrefillRows * D * 2;
     uint8_t* sV = sK + T * D * 2;
@@ -375,7 +389,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const Prefi
             const int t0 = k * T;
             const int valid = min(T, Ls - t0);
             // keys first: S of this tile can start while the values are dequantised
-            dequant_tile<KK, D>(st, st + p.st_ks, sK, T, valid, tid);
+            dequant_tile<KK, D>(st, st + p.st_ks, sK, T, lgT, valid, tid);
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncthreads();
             if (tid == 0) {
@@ -390,7 +404,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const Prefi
                 wait_or_flag(barO, (rnd - 1) & 1u);
                 tc::fence_after();
             }
-            dequant_tile<KV, D>(st + p.st_vc, st + p.st_vs, sV, T, valid, tid);
+            dequant_tile<KV, D>(st + p.st_vc, st + p.st_vs, sV, T, lgT, valid, tid);
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 
             // ---- scores of this thread's row, columns [32 h, 32 h + 32) of the tile
