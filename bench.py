@@ -55,13 +55,19 @@ HEADLINE_TRAFFIC = {"bytes": 125_782_016 + 3_462_400,
 KERNEL_SOURCES = ("kvq_decode.cu", "kvq_common.cuh", "kvq_quant.cuh", "kvq_internal.h")
 
 
-def kernel_digest() -> str:
-    """sha256 of the decode kernel's sources with comments and whitespace
-    removed: edits to comments keep a recorded capture valid, code edits void it."""
+# The same for the chunked-prefill kernel on its workload.
+PREFILL_TRAFFIC = {"bytes": 175_584_768 + 42_600_960,
+                   "sources_sha256": "8018ed37346010a003d7008da643f155893e94e2f5dc68613458ca8b46a53099"}
+PREFILL_SOURCES = ("kvq_prefill.cu", "kvq_prefill.h", "kvq_tc.cuh", "kvq_common.cuh")
+
+
+def kernel_digest(files=KERNEL_SOURCES) -> str:
+    """sha256 of a kernel's sources with comments and whitespace removed:
+    edits to comments keep a recorded capture valid, code edits void it."""
     import hashlib
     import re
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
+    for f in files:
         with open(os.path.join(ROOT, "quantized_paged_kv_03_b200", "csrc", f)) as fh:
             src = fh.read()
         src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
@@ -75,6 +81,11 @@ def headline_traffic(config: int, batch) -> int | None:
     if config != HEADLINE_CONFIG or batch is not None:
         return None
     return HEADLINE_TRAFFIC["bytes"] if kernel_digest() == HEADLINE_TRAFFIC["sources_sha256"] else None
+
+
+def prefill_traffic() -> int | None:
+    ok = kernel_digest(PREFILL_SOURCES) == PREFILL_TRAFFIC["sources_sha256"]
+    return PREFILL_TRAFFIC["bytes"] if ok else None
 
 
 def load_peaks():
@@ -384,7 +395,8 @@ class PrefillArm:
             "append_GBps": round(self.app_bytes / (app_ms * 1e-3) / 1e9, 1),
             "flops_per_launch": self.flops, "kv_bytes": self.kv_bytes,
             "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": peak_tflops,
-                         "unit": "TFLOP/s", "frac": round(tflops / peak_tflops, 4), "traffic": None,
+                         "unit": "TFLOP/s", "frac": round(tflops / peak_tflops, 4), "traffic": prefill_traffic(),
+                         "traffic_unit": "bytes per launch (ncu dram read + write)",
                          "kernel": "prefill_kernel (tcgen05.mma kind::f16, fp32 accumulation in tensor memory)",
                          "peak_source": f"{peak_kind} bf16_tflops (fp16 has the same dense rate)"},
             "gpu_launches_per_step": 2,
