@@ -5,9 +5,12 @@ decode attention over every sequence's cache (all steps of the hot path), with
 the prefix already in the cache and all inputs resident in HBM.  The headline
 workload is INT8-G64 (batch 8, lengths uniform in [1024, 8192], 8 kv-heads,
 32 query heads, head_dim 256, 64-token pages); the other formats' workloads are
-reported under "formats".
+reported under "formats", and the chunked-prefill workload (append a 512-token
+chunk per sequence + causal attention of its queries, against the tensor-core
+roofline) under "prefill".
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--quick]
+                    [--prefill-only]
 
 N > 1: launched by torchrun, one rank per GPU; every rank runs its own replica
 (the path has no exchange step), timings are the max over ranks.

@@ -1,4 +1,4 @@
-"""Seeded synthetic inputs for the KV-cache append + decode path.
+"""Seeded synthetic inputs for the KV-cache append, decode and chunked-prefill paths.
 
 This module draws random numbers and shapes them; it holds none of the
 method's arithmetic (no rotation, no scales, no codes).  Tests feed the same
@@ -16,7 +16,9 @@ dataset for this path):
   * block tables: each sequence's pages are a slice of one random permutation
     of the page pool, so consecutive pages are not adjacent in memory;
   * the last token of every sequence is the step's new token (appended during
-    the step, then attended to); the others are the prefix.
+    the step, then attended to); the others are the prefix;
+  * chunked prefill: the last n tokens of a sequence are the chunk, its query
+    rows N(0, 1) bf16 like the decode queries (``prefill_queries``).
 Every stream is a child of ``SeedSequence([seed, stream_id, ...])`` so results do
 not depend on the thread count.
 """
