@@ -637,6 +637,13 @@ def main():
         tpk, tkind = load_tensor_peak()
         pa = PrefillArm(seed_offset=rank)
         prefill = pa.report(args.steps, args.warmup, flush, tpk, tkind)
+        if dist is not None:
+            # whole job: every rank's chunk over the slowest rank's time
+            att_tf, att_ms = whole_job_rate(pa.flops / 1e12, prefill["attention_ms"], dist)
+            tok_s, step_ms = whole_job_rate(pa.chunk_tokens, prefill["step_ms"], dist)
+            prefill.update(attention_ms=round(att_ms, 5), attention_TFLOPs=round(att_tf, 1),
+                           step_ms=round(step_ms, 5), chunk_tokens_per_s=round(tok_s, 1),
+                           scope=f"whole job, {world} replicas; roofline per GPU")
         del pa
         torch.cuda.empty_cache()
 
