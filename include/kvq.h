@@ -40,7 +40,7 @@
 extern "C" {
 #endif
 
-#define KVQ_VERSION 1
+#define KVQ_VERSION 2   /* 2: kvq_prefill_attention */
 
 typedef enum {
     KVQ_OK = 0,

@@ -33,7 +33,7 @@ def test_library_exports_every_declared_symbol(L):
     for n in names:
         assert hasattr(L, n), n
     assert sorted(K.exported_symbols()) == names
-    assert L.kvq_version() == 1
+    assert L.kvq_version() == 2
 
 
 def test_token_bytes_table(L):
