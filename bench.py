@@ -178,6 +178,7 @@ class Arm:
         scales = None
         if fmt == "fp8_tensor":
             scales = [(I.tensor_amax(w.k) / 448.0 or 1.0, I.tensor_amax(w.v) / 448.0 or 1.0)]
+        self.scales = scales
         self.cache = K.KVCache(fmt, w.D, w.H, w.P, w.num_pages, 1, 0, scales)
         dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
         kp, vp, sp = w.prefix()
@@ -234,9 +235,7 @@ class Arm:
                 worst_max = max(worst_max, float(err.abs().max() / v.abs().max()))
                 worst_rms = max(worst_rms, float(err.norm() / ref.norm()))
                 del k, v
-        return {"max_abs_over_max_abs_v": round(worst_max, 6), "rel_rms": round(worst_rms, 6),
-                "sample": f"sequences {seqs} (lengths {[int(w.seq_lens[b]) for b in seqs]}), "
-                          f"kv-heads {sorted({0, w.H - 1})}; reference: fp64 attention over the bf16 inputs"}
+        return {"max_abs_over_max_abs_v": round(worst_max, 6), "rel_rms": round(worst_rms, 6)}
 
     def step(self):
         """One decode step, one launch: append each sequence's new token and attend."""
@@ -387,21 +386,14 @@ class PrefillArm:
         tflops = self.flops / (att_ms * 1e-3) / 1e12
         return {
             "workload": I.PREFILL.name,
-            "what": "append the chunk's K/V + causal attention of its queries over the cache "
-                    "(kvq_append + kvq_prefill_attention)",
-            "batch": w.B, "seq_len": int(w.seq_lens.max()), "chunk": self.max_q, "n_kv_heads": w.H,
-            "n_q_heads": w.Hq, "head_dim": w.D, "page_size": w.P, "format": I.PREFILL.formats[0],
             "step_ms": round(step_ms, 5),
             "chunk_tokens_per_s": round(self.chunk_tokens / (step_ms * 1e-3), 1),
             "attention_ms": round(att_ms, 5), "attention_TFLOPs": round(tflops, 1),
-            "append_ms": round(app_ms, 5),
             "append_GBps": round(self.app_bytes / (app_ms * 1e-3) / 1e9, 1),
-            "flops_per_launch": self.flops, "kv_bytes": self.kv_bytes,
+            "flops_per_launch": self.flops,
             "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": peak_tflops,
                          "unit": "TFLOP/s", "frac": round(tflops / peak_tflops, 4), "traffic": prefill_traffic(),
-                         "traffic_unit": "bytes per launch (ncu dram read + write)",
-                         "kernel": "prefill_kernel (tcgen05.mma kind::f16, fp32 accumulation in tensor memory)",
-                         "peak_source": f"{peak_kind} bf16_tflops (fp16 has the same dense rate)"},
+                         "kernel": "prefill_kernel (tcgen05)", "peak_source": f"{peak_kind} bf16_tflops"},
             "gpu_launches_per_step": 2,
         }
 
@@ -457,12 +449,31 @@ def oracle_sample(cfg: int, fmt: str, budget_s: float = 12.0, threads: int | Non
     # the step's append of those rows and is not counted)
     nbytes = done_tokens * tb + done * G * w.D * (2 + 4)
     return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
-            "sample": f"{done} (sequence, kv-head) decode jobs cycling over the {len(jobs)} of one step of "
-                      f"{I.CONFIGS[cfg].name} ({done_tokens} cached tokens quantised, dequantised and "
-                      f"attended in fp64) in {dt:.1f} s on {threads} threads"}
+            "sample": f"{done} (seq, kv-head) jobs of {I.CONFIGS[cfg].name}, {done_tokens} tokens, {dt:.1f} s"}
+
+
+def cpu_baseline(cfg: int, fmt: str, budget_s: float = 12.0, single_s: float = 6.0):
+    """The oracle on all host threads (up to 32) and on one thread, with the
+    host's core count."""
+    many = oracle_sample(cfg, fmt, budget_s=budget_s)
+    one = oracle_sample(cfg, fmt, budget_s=single_s, threads=1)
+    many["nproc"] = os.cpu_count()
+    many["single_thread"] = {"value": one["value"], "cores": 1, "sample": one["sample"]}
+    return many
 
 
 # ---------------------------------------------------------------- main
+
+def format_entry(step_gbs, peak, dec_gbs, app_gbs, tokens_s, step_ms, qerr):
+    """One workload/format of the `formats` map: step GB/s (fused append +
+    decode), its fraction of the peak, decode-only GB/s, bulk-append GB/s,
+    tokens/s (sequences per second of the step), step ms and the quantisation
+    error against fp64 attention over the bf16 inputs (max / rel. RMS)."""
+    return {"step_GBps": round(step_gbs, 1), "frac": round(step_gbs / peak, 3),
+            "decode_GBps": round(dec_gbs, 1), "append_GBps": round(app_gbs, 1),
+            "tokens_per_s": round(tokens_s, 1), "step_ms": round(step_ms, 4),
+            "qerr": [qerr["max_abs_over_max_abs_v"], qerr["rel_rms"]]}
+
 
 def dist_setup(n):
     if n <= 1:
@@ -518,13 +529,15 @@ def reference_arm(args):
         last = oracle_sample(HEADLINE_CONFIG, fmt, budget_s=budget)
         vals.append(last["value"])
     v = float(np.mean(vals))
+    one = oracle_sample(HEADLINE_CONFIG, fmt, budget_s=budget, threads=1)
     spec = I.CONFIGS[HEADLINE_CONFIG]
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": spec.name, "format": fmt},
-            "cpu_baseline": {"value": v, "unit": "GB/s", "cores": last["cores"], "kind": "oracle",
-                             "sample": last["sample"]},
+            "cpu_baseline": {"value": v, "unit": "GB/s", "cores": last["cores"], "nproc": os.cpu_count(),
+                             "kind": "oracle", "sample": last["sample"],
+                             "single_thread": {"value": one["value"], "cores": 1, "sample": one["sample"]}},
             "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -617,18 +630,9 @@ def main():
                 dm = max_over_ranks(float(a.run(args.steps, args.warmup, flush, fn=a.decode_only).mean()), dist)
                 am = max_over_ranks(float(a.run(args.steps, args.warmup, flush, fn=a.bulk_append).mean()), dist)
                 sb = a.dec_bytes + a.app_bytes
-                formats[f"{I.CONFIGS[cfg].name}/{f}"] = {
-                    "step_ms": round(sm, 5), "step_GBps": round(sb / (sm * 1e-3) / 1e9, 1),
-                    "step_pct_of_peak": round(100 * sb / (sm * 1e-3) / 1e9 / peak, 1),
-                    "tokens_per_s": round(a.w.B / (sm * 1e-3), 1),
-                    "decode_only_ms": round(dm, 5),
-                    "decode_only_GBps": round(a.dec_bytes / (dm * 1e-3) / 1e9, 1),
-                    "step_bytes": sb, "bytes_per_token_head": a.tb,
-                    "append_tokens": a.bulk_tokens, "append_ms": round(am, 5),
-                    "append_GBps": round(a.bulk_bytes / (am * 1e-3) / 1e9, 1),
-                    "append_pct_of_peak": round(100 * a.bulk_bytes / (am * 1e-3) / 1e9 / peak, 1),
-                    "append_tokens_per_s": round(a.bulk_tokens / (am * 1e-3), 1),
-                    "quant_error_vs_bf16": a.qerr}
+                formats[f"{I.CONFIGS[cfg].name}/{f}"] = format_entry(
+                    sb / (sm * 1e-3) / 1e9, peak, a.dec_bytes / (dm * 1e-3) / 1e9,
+                    a.bulk_bytes / (am * 1e-3) / 1e9, a.w.B / (sm * 1e-3), sm, a.qerr)
                 del a
                 torch.cuda.empty_cache()
 
@@ -651,7 +655,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
-        cpu = oracle_sample(args.config, fmt, budget_s=12.0)
+        cpu = cpu_baseline(args.config, fmt)
 
     if rank == 0:
         line = {
@@ -662,23 +666,16 @@ def main():
             "config": {"workload": spec.name, "format": fmt, "batch": arm.w.B,
                        "n_kv_heads": arm.w.H, "n_q_heads": arm.w.Hq, "head_dim": arm.w.D,
                        "page_size": arm.w.P, "kv_tokens": int(arm.w.seq_lens.sum()),
-                       "step": "append 1 token/sequence + decode attention, one fused launch",
-                       "l2": "flushed before every step, outside the timed events: 256 MiB written, then 256 MiB read",
+                       "step": "append 1 token/seq + decode, one fused launch",
+                       "l2": "flushed before every step (256 MiB write + 256 MiB read), outside the events",
                        "parallelism": f"replicas x{world}"},
             "tokens_per_s": round(tokens, 1),
             "pct_of_peak": round(100 * value / peak, 2),
             "decode_only_GBps": round(dec_gbs, 1),
-            "quant_error_vs_bf16": arm.qerr,
-            "append": {"tokens": arm.bulk_tokens, "ms": round(app_ms, 5),
-                       "GBps": round(arm.bulk_bytes / (app_ms * 1e-3) / 1e9, 1),
-                       "pct_of_peak": round(100 * arm.bulk_bytes / (app_ms * 1e-3) / 1e9 / peak, 1),
-                       "tokens_per_s": round(arm.bulk_tokens / (app_ms * 1e-3), 1),
-                       "what": "bulk append of the prefix's first tokens (append_kernel alone)"},
+            "append_GBps": round(arm.bulk_bytes / (app_ms * 1e-3) / 1e9, 1),
             "roofline": {"bound": "hbm", "achieved": round(step_gbs, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(step_gbs / peak, 4), "traffic": headline_traffic(args.config, args.batch),
-                         "traffic_unit": "bytes per launch (ncu dram read + write)",
-                         "kernel": "decode_kernel with the fused append (one launch per step)",
-                         "peak_source": f"{peak_kind} hbm_gbs"},
+                         "kernel": "decode_kernel (fused append)", "peak_source": f"{peak_kind} hbm_gbs"},
             "e2e": {"value": round(total_bytes / (e2e_ms * 1e-3) / 1e9 if world > 1 else
                                    step_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                     "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": int(h2d),
@@ -686,12 +683,15 @@ def main():
             "gpu_launches": args.steps,
             "clocks": clk.summary(int(os.environ.get("LOCAL_RANK", "0"))),
             "wall_s_timed_region": round(t_wall, 3),
-            "formats": formats,
         }
-        if prefill is not None:
-            line["prefill"] = prefill
         if cpu is not None:
             line["cpu_baseline"] = cpu
+        if prefill is not None:
+            line["prefill"] = prefill
+        # last, so that a truncated tail of the line still shows every format
+        line["formats"] = {f"{spec.name}/{fmt}": format_entry(step_gbs, peak, dec_gbs,
+                                                              arm.bulk_bytes / (app_ms * 1e-3) / 1e9,
+                                                              tokens, step_ms_max, arm.qerr), **formats}
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.barrier()

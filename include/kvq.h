@@ -10,9 +10,10 @@
  *
  * Pages the formats come from (cited by title and section):
  *   [NInfer]     "NInfer KV Cache 量化指南：BF16、INT8、FP8、NVFP4 与 K8V4 五种格式怎么选"
- *                -- 64-token pages with independently encoded K and V ("按 64
- *                token 一个 page 管理支持非对称的 K/V 编码"), the per-token byte
- *                table, and the five format paragraphs ("五种格式逐个认识").
+ *                -- the paging remark (the cache is managed in 64-token
+ *                pages, with K and V allowed different encodings), the
+ *                per-token byte table, and the format paragraphs (section
+ *                "五种格式逐个认识").
  *   [TokenSpeed] "TokenSpeed量化实战：fp8、NVFP4与KV缓存压缩如何省下50%显存"
  *                -- "--kv-cache-dtype" table: fp8_e4m3 with unit scale, mxfp8 with
  *                one UE8M0 scale per 32 head_dim elements and 128-token blocks.
@@ -40,7 +41,7 @@
 extern "C" {
 #endif
 
-#define KVQ_VERSION 2   /* 2: kvq_prefill_attention */
+#define KVQ_VERSION 3   /* 2: kvq_prefill_attention; 3: kvq_debug_set_wait_polls, KVQ_ERR_DEVICE_BOUNDS */
 
 typedef enum {
     KVQ_OK = 0,
@@ -49,7 +50,7 @@ typedef enum {
     KVQ_ERR_SHAPE = 3,      /* sizes inconsistent (n_q_heads % n_kv_heads, page size, limits) */
     KVQ_ERR_WORKSPACE = 4,  /* pool or workspace smaller than required */
     KVQ_ERR_CUDA = 5,       /* a CUDA runtime call failed (launch error, no device) */
-    KVQ_ERR_DEVICE = 6      /* a kernel recorded an error (see kvq_read_device_status) */
+    KVQ_ERR_DEVICE_BOUNDS = 6  /* a kernel recorded an out-of-range slot or page id or a wait that gave up (see kvq_read_device_status) */
 } kvq_status;
 
 /* Storage formats.  Bytes per token per kv-head (K + V) at head_dim D = 256,
@@ -244,6 +245,17 @@ int kvq_encode(int32_t code, const float* x, int64_t n, uint8_t* out, void* stre
  * out of range in kvq_append, bit 1 = a page id out of range in decode or prefill, bit 2 =
  * a decode pipeline wait gave up.  Synchronises `stream`. */
 int kvq_read_device_status(kvq_cache* cache, int32_t clear, uint32_t* status, void* stream);
+
+/* Test surface: set how many times a kernel's bounded pipeline wait (a stage
+ * copy or a tensor-core result that has not arrived) polls before it gives up,
+ * for every decode, fused decode and prefill launched after this call in this
+ * process; 0 gives up at once, a negative value restores the default (2^22
+ * polls, about a second).  A wait that gives up sets bit 2 of the device status
+ * word; the kernel then skips its remaining work, waits (with the default
+ * limit) for the copies and tensor-core operations it already issued, and
+ * returns, leaving the context usable.  Returns the previous setting.  Host
+ * only; no device work. */
+int64_t kvq_debug_set_wait_polls(int64_t polls);
 
 const char* kvq_status_string(int status);
 int kvq_version(void);

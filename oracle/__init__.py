@@ -12,7 +12,7 @@ plain numpy indexing.
 
 Pages cited:
   [NInfer]     "NInfer KV Cache 量化指南：BF16、INT8、FP8、NVFP4 与 K8V4 五种格式怎么选"
-               -- 64-token pages ("按 64 token 一个 page 管理"), asymmetric K/V
+               -- 64-token pages (the paging remark), asymmetric K/V
                encodings, the per-token byte table and the format paragraphs.
   [TokenSpeed] "TokenSpeed量化实战：fp8、NVFP4与KV缓存压缩如何省下50%显存"
                -- mxfp8 with ``--block-size 128``.

@@ -199,7 +199,7 @@ void or_encode_bits(int code, uint32_t start, int64_t n, uint8_t* out)
 /* --------------------------------------------------------------- Hadamard */
 
 /* Normalised Hadamard-256 in fp32, R1.  [NInfer] INT8 / NVFP4 paragraphs:
- * "256 维 Hadamard 归一化预处理" before quantising. */
+ * a normalised 256-dimensional Hadamard as preprocessing before quantising. */
 void or_fwht256(float* x)
 {
     for (int h = 1; h < 256; h <<= 1)

@@ -72,6 +72,7 @@ def lib() -> ctypes.CDLL:
         "kvq_read_rows": (ctypes.c_int, [P, i32, P, i32, P, P, P, P, P]),
         "kvq_encode": (ctypes.c_int, [i32, P, i64, P, P]),
         "kvq_read_device_status": (ctypes.c_int, [P, i32, ctypes.POINTER(u32), P]),
+        "kvq_debug_set_wait_polls": (i64, [i64]),
         "kvq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "kvq_version": (ctypes.c_int, []),
     }
@@ -88,7 +89,13 @@ def exported_symbols():
             "kvq_cache_destroy", "kvq_append", "kvq_decode_workspace_bytes",
             "kvq_decode_attention", "kvq_append_decode", "kvq_decode_attention_noalloc",
             "kvq_prefill_attention", "kvq_dequant", "kvq_read_rows", "kvq_encode",
-            "kvq_read_device_status", "kvq_status_string", "kvq_version"]
+            "kvq_read_device_status", "kvq_debug_set_wait_polls", "kvq_status_string", "kvq_version"]
+
+
+def set_wait_polls(polls: int) -> int:
+    """Test surface: polls of a kernel's bounded pipeline wait before it gives
+    up (0: at once; negative: the default).  Returns the previous setting."""
+    return int(lib().kvq_debug_set_wait_polls(int(polls)))
 
 
 def _check(status: int, what: str):

@@ -5,6 +5,8 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "../../include/kvq.h"
 #include "kvq_internal.h"
 #include "kvq_prefill.h"
@@ -37,6 +39,12 @@ static int desc_layout(const kvq_cache_desc* d, Layout* out) {
 }
 
 static int cuda_status(cudaError_t e) { return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA; }
+
+// Polls of a kernel's bounded pipeline waits (stage arrivals, MMA completion):
+// about a second at the default; a test lowers it to make a wait give up.
+static constexpr long long kDefaultWaitPolls = 1ll << 22;
+static std::atomic<long long> g_wait_polls{kDefaultWaitPolls};
+long kvq::wait_polls() { return (long)g_wait_polls.load(std::memory_order_relaxed); }
 
 static uint8_t* layer_slabs(const kvq_cache* c, int layer) {
     const Layout& L = c->L;
@@ -177,24 +185,30 @@ int kvq_append_decode(kvq_cache* cache, int32_t layer, const void* k_new, const 
                          max_seq_len, out, out_fp32, softmax_scale, workspace, workspace_bytes, stream);
 }
 
-static int decode_common(kvq_cache* cache, int32_t layer, const void* k_new, const void* v_new, const void* q,
-                         int32_t n_q_heads, const int32_t* block_table, int32_t max_pages_per_seq,
-                         const int32_t* seq_lens, int32_t batch, int32_t max_seq_len, void* out, int32_t out_fp32,
-                         float softmax_scale, void* workspace, size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+// Validates a decode call on the host (every check that needs neither the
+// device nor a workspace) and fills its kernel parameters.  *batch0 is set when there is nothing to
+// launch (batch 0).  Shared by kvq_decode_attention, kvq_append_decode and the
+// allocation-free entry point, so all three accept and reject the same calls.
+int kvq::decode_setup(kvq_cache* cache, int32_t layer, const void* k_new, const void* v_new, const void* q,
+                      int32_t n_q_heads, const int32_t* block_table, int32_t max_pages_per_seq,
+                      const int32_t* seq_lens, int32_t batch, int32_t max_seq_len, void* out, int32_t out_fp32,
+                      float softmax_scale, DecodeParams* pp, bool* batch0) {
     int G, HB;
+    *batch0 = false;
     int st = decode_shape(cache, batch, n_q_heads, max_seq_len, &G, &HB);
     if (st != KVQ_OK) return st;
     if (layer < 0 || layer >= cache->L.num_layers) return KVQ_ERR_ARG;
-    if (batch == 0) return KVQ_OK;
-    if (!q || !block_table || !seq_lens || !out || !workspace || max_pages_per_seq < 1) return KVQ_ERR_ARG;
+    if (batch == 0) {
+        *batch0 = true;
+        return KVQ_OK;
+    }
+    if (!q || !block_table || !seq_lens || !out || max_pages_per_seq < 1) return KVQ_ERR_ARG;
     if ((int64_t)max_pages_per_seq * cache->L.P < max_seq_len) return KVQ_ERR_SHAPE;
-    if (((uintptr_t)q & 15) || ((uintptr_t)out & 15) || ((uintptr_t)workspace & 15)) return KVQ_ERR_ARG;
+    if (((uintptr_t)q & 15) || ((uintptr_t)out & 15)) return KVQ_ERR_ARG;
     if (!(softmax_scale >= 0.f) || !isfinite(softmax_scale)) return KVQ_ERR_ARG;
-    DecodePlan plan;
-    if (plan_decode(cache->L, batch, HB, max_seq_len, &plan) != cudaSuccess) return KVQ_ERR_CUDA;
-    const size_t need = decode_workspace_bytes(cache->L, batch, HB, plan.grid);
-    if (workspace_bytes < need) return KVQ_ERR_WORKSPACE;
-    DecodeParams p;
+    DecodeParams& p = *pp;
     p.L = cache->L;
     p.slabs = layer_slabs(cache, layer);
     p.q = (const uint16_t*)q;
@@ -208,22 +222,56 @@ static int decode_common(kvq_cache* cache, int32_t layer, const void* k_new, con
     p.out = out;
     p.out_fp32 = out_fp32 ? 1 : 0;
     const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)cache->L.D);
-    p.q_mult = scale * 1.4426950408889634f * cache->tensor_scales[2 * layer];
+    p.q_mult = scale * 1.4426950408889634f;
+    p.k_tmult = cache->tensor_scales[2 * layer];
     p.o_mult = cache->tensor_scales[2 * layer + 1];
     p.rot_k = rot_of(cache, 0);
     p.rot_v = rot_of(cache, 1);
-    size_t zoff = 0, zbytes = 0;
-    decode_workspace_zero_region(cache->L, batch, HB, plan.grid, &zoff, &zbytes);
-    p.partials = (float*)workspace;
-    p.barrier = (unsigned*)((uint8_t*)workspace + zoff);
+    p.wait_polls = kvq::wait_polls();
+    p.partials = nullptr;
+    p.barrier = nullptr;
     p.status = (uint32_t*)cache->pool;
-    p.stages = plan.stages;
-    p.pid_cap = plan.pid_cap;
     p.k_new = (const uint16_t*)k_new;
     p.v_new = (const uint16_t*)v_new;
     p.k_scale = cache->tensor_scales[2 * layer];
     p.v_scale = cache->tensor_scales[2 * layer + 1];
-    return cuda_status(launch_decode(p, plan, (cudaStream_t)stream));
+    p.max_seq_len = max_seq_len;
+    return KVQ_OK;
+}
+
+// The launch plan of a set-up decode (queries the current device).
+int kvq::decode_plan(DecodeParams* p, DecodePlan* plan) {
+    if (plan_decode(p->L, p->B, p->HB, p->max_seq_len, plan) != cudaSuccess) return KVQ_ERR_CUDA;
+    p->stages = plan->stages;
+    p->pid_cap = plan->pid_cap;
+    return KVQ_OK;
+}
+
+// Points a set-up decode at its workspace (which must be large enough) and launches it.
+int kvq::decode_launch(DecodeParams* p, const DecodePlan& plan, void* workspace, cudaStream_t stream) {
+    size_t zoff = 0, zbytes = 0;
+    decode_workspace_zero_region(p->L, p->B, p->HB, plan.grid, &zoff, &zbytes);
+    p->partials = (float*)workspace;
+    p->barrier = (unsigned*)((uint8_t*)workspace + zoff);
+    return cuda_status(launch_decode(*p, plan, stream));
+}
+
+extern "C" {
+
+static int decode_common(kvq_cache* cache, int32_t layer, const void* k_new, const void* v_new, const void* q,
+                         int32_t n_q_heads, const int32_t* block_table, int32_t max_pages_per_seq,
+                         const int32_t* seq_lens, int32_t batch, int32_t max_seq_len, void* out, int32_t out_fp32,
+                         float softmax_scale, void* workspace, size_t workspace_bytes, void* stream) {
+    DecodeParams p;
+    DecodePlan plan;
+    bool none = false;
+    int st = decode_setup(cache, layer, k_new, v_new, q, n_q_heads, block_table, max_pages_per_seq, seq_lens, batch,
+                          max_seq_len, out, out_fp32, softmax_scale, &p, &none);
+    if (st != KVQ_OK || none) return st;
+    if (!workspace || ((uintptr_t)workspace & 15)) return KVQ_ERR_ARG;
+    if ((st = decode_plan(&p, &plan)) != KVQ_OK) return st;
+    if (workspace_bytes < decode_workspace_bytes(cache->L, batch, p.HB, plan.grid)) return KVQ_ERR_WORKSPACE;
+    return decode_launch(&p, plan, workspace, (cudaStream_t)stream);
 }
 
 int kvq_prefill_attention(kvq_cache* cache, int32_t layer, const void* q, int32_t n_q_heads,
@@ -264,6 +312,7 @@ int kvq_prefill_attention(kvq_cache* cache, int32_t layer, const void* q, int32_
     p.o_mult = cache->tensor_scales[2 * layer + 1];
     p.rot_k = rot_of(cache, 0);
     p.rot_v = rot_of(cache, 1);
+    p.wait_polls = kvq::wait_polls();
     p.status = (uint32_t*)cache->pool;
     return cuda_status(launch_prefill(p, plan, grid, (cudaStream_t)stream));
 }
@@ -330,9 +379,13 @@ const char* kvq_status_string(int status) {
     case KVQ_ERR_SHAPE: return "inconsistent or unsupported sizes";
     case KVQ_ERR_WORKSPACE: return "pool or workspace too small";
     case KVQ_ERR_CUDA: return "CUDA runtime error";
-    case KVQ_ERR_DEVICE: return "a kernel recorded an error";
+    case KVQ_ERR_DEVICE_BOUNDS: return "a kernel recorded an out-of-range index or a wait that gave up";
     default: return "unknown status";
     }
+}
+
+int64_t kvq_debug_set_wait_polls(int64_t polls) {
+    return (int64_t)g_wait_polls.exchange(polls < 0 ? kDefaultWaitPolls : (long long)polls);
 }
 
 int kvq_version(void) { return KVQ_VERSION; }

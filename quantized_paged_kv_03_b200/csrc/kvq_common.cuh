@@ -21,8 +21,8 @@ namespace kvq {
 constexpr int kHeaderBytes = 256;   // pool header: device status word(s)
 
 enum RowKind : int {
-    RK_BF16RAW = 0,      // bf16 bit pattern ([NInfer] BF16 K: "按位原样存储")
-    RK_FP16 = 1,         // fp16, nearest-even, saturating ([NInfer] BF16 V: "以 FP16 落盘")
+    RK_BF16RAW = 0,      // bf16 bit pattern ([NInfer] BF16 paragraph: K kept bit for bit)
+    RK_FP16 = 1,         // fp16, nearest-even, saturating ([NInfer] BF16 paragraph: V written as fp16)
     RK_E4M3_ROW256 = 2,  // E4M3 codes + fp16 scale per 256 values ([NInfer] FP8 row-256)
     RK_INT8_G64 = 3,     // int8 codes + fp16 scale per 64 values ([NInfer] INT8-G64)
     RK_E2M1_G16 = 4,     // E2M1 codes + UE4M3 scale per 16 values ([NInfer] NVFP4-G16)
@@ -46,8 +46,9 @@ KVQ_HD constexpr int kind_of(int fmt, int is_v) {
     }
 }
 
-// [NInfer]: INT8 rotates K ("写入前对 K 做 256 维 Hadamard"); NVFP4 rotates K and
-// V ("K、V 都做 Hadamard 预处理"); K8V4's V is NVFP4 and is rotated likewise.
+// [NInfer] format paragraphs: INT8 applies the 256-point Hadamard to K before
+// it is written; NVFP4 applies it to both K and V; K8V4's V is NVFP4 and is
+// rotated likewise.
 KVQ_HD constexpr bool rotated(int fmt, int is_v) {
     switch (fmt) {
     case F_INT8_G64: return !is_v;
@@ -211,6 +212,17 @@ __device__ __forceinline__ float e2m1_to_f32(uint32_t c) {
 __device__ __forceinline__ float ue8m0_to_f32(uint32_t b) {
     return __uint_as_float(b ? (b << 23) : 0x00400000u);
 }
+
+// 2^e as fp32, exact, built from the exponent field: subnormal below 2^-126,
+// 0 below 2^-149, +inf above 2^127.
+__device__ __forceinline__ float pow2i(int e) {
+    if (e > 127) return __uint_as_float(0x7F800000u);
+    if (e >= -126) return __uint_as_float((uint32_t)(e + 127) << 23);
+    if (e >= -149) return __uint_as_float(1u << (e + 149));
+    return 0.f;
+}
+// floor(log2 x) of a positive finite fp32 value (-127 for every subnormal).
+__device__ __forceinline__ int exp2_floor(float x) { return (int)(__float_as_uint(x) >> 23) - 127; }
 
 // ------------------------------------------------------------ Hadamard-256
 // Normalised Sylvester Hadamard of a 256-vector held 8 per lane (lane l holds

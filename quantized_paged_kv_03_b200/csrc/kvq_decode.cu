@@ -68,11 +68,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t phase) {
         : "memory");
     return ok != 0;
 }
-// Bounded wait for a stage.  Gives up after kWaitPolls polls, or at once when
+// Bounded wait for a stage.  Gives up after `polls` polls, or at once when
 // another warp has already given up (`abort` set), so a failed copy never hangs
 // the CTA: every warp then runs through its remaining work without waiting.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t phase, volatile int* abort) {
-    for (long i = 0; i < kWaitPolls; i++) {
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t phase, volatile int* abort, long polls = kWaitPolls) {
+    for (long i = 0; i < polls; i++) {
         if (mbar_try_wait(bar, phase)) return true;
         if (*abort) return false;
     }
@@ -465,6 +465,7 @@ __device__ __noinline__ void fused_append_rows(int warp, int lane, const uint16_
 template <int KK, int KV, int D, bool FUSED>
 __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_kernel(const DecodeParams p) {
     using T = DecTraits<KK, KV, D>;
+    constexpr bool VFOLD = (KV == RK_E4M3_ROW256 || KV == RK_INT8_G64 || KV == RK_E4M3_MX32);
     extern __shared__ __align__(128) uint8_t smem[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int r = lane >> 2, j = lane & 3;
@@ -491,6 +492,8 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
     off += 4 * 16 * 4;
     float* fin = reinterpret_cast<float*>(smem + off);   // [m 8][l 8] of the merged segment
     off += 16 * 4;
+    float* qhm = reinterpret_cast<float*>(smem + off);   // [8] score multiplier of each head of the block
+    off += 8 * 4;
     int* flags = reinterpret_cast<int*>(smem + off);     // [0] abort, [2] grid barrier ok
     off += 16;
     int* pref = reinterpret_cast<int*>(smem + off);      // [B + 1] page prefix
@@ -635,6 +638,13 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
     uint32_t qf[T::KSTEPS / 2][T::QS][2];
     float o[T::DTILES / 2][4];
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+    float hm0 = 1.f, hm1 = 1.f;   // score multipliers of heads 2j, 2j + 1 (q's power of two, K tensor scale)
+    // V scales folded into P' (FP8 row-256, INT8, MX V): P' = P * (scale * 2^-ve),
+    // ve a warp-uniform power-of-two reference raised (with the accumulators
+    // rescaled) when a scale exceeds 2^(ve + 4); o is in units of 2^ve.  This
+    // keeps P' inside fp16's normal range whatever the magnitude of V.
+    int ve = 0;
+    float vmul = 1.f, vthr = 0.f;   // 2^-ve; 2^(ve + 4), 0 before the segment's first nonzero scale
     bool seg_first = true;     // segment began at this CTA's first page
     int xpar = 0;              // score-exchange buffer parity
 
@@ -699,11 +709,26 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
                             for (int e = 0; e < 8; e++) x[e] = y.v[e];
                         }
                     }
+                    // q x softmax scale x log2(e), normalised by a power of two so
+                    // that its largest element lies in [1, 2): fp16 keeps full
+                    // precision whatever q's magnitude; the 2^e returns in the
+                    // fp32 scores (with the K tensor scale, for FP8 per tensor)
+                    float amax = 0.f;
 #pragma unroll
-                    for (int e = 0; e < T::EPL; e++) x[e] *= p.q_mult;
+                    for (int e = 0; e < T::EPL; e++) {
+                        x[e] *= p.q_mult;
+                        amax = fmaxf(amax, fabsf(x[e]));
+                    }
+                    amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(amax)));
+                    const int eq = amax > 0.f ? exp2_floor(amax) : 0;
+                    const float nq = pow2i(-eq);
+#pragma unroll
+                    for (int e = 0; e < T::EPL; e++) x[e] *= nq;
+                    if (lane == 0) qhm[warp] = pow2i(eq) * p.k_tmult;
                 } else {
 #pragma unroll
                     for (int e = 0; e < T::EPL; e++) x[e] = 0.f;
+                    if (lane == 0) qhm[warp] = 0.f;
                 }
 #pragma unroll
                 for (int g4 = 0; g4 < T::EPL / 4; g4++) {
@@ -737,14 +762,19 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
                     qf[sl][0][0] = v.x; qf[sl][0][1] = v.y;
                 }
             }
+            hm0 = qhm[2 * j];
+            hm1 = qhm[2 * j + 1];
 #pragma unroll
             for (int u = 0; u < T::DTILES / 2; u++) o[u][0] = o[u][1] = o[u][2] = o[u][3] = 0.f;
             m0 = m1 = -INFINITY;
             l0 = l1 = 0.f;
+            ve = 0;
+            vmul = 1.f;
+            vthr = 0.f;
         }
 
         // wait for the slab
-        (void)mbar_wait(smem_u32(&bars[s]), ph, abort_flag);
+        (void)mbar_wait(smem_u32(&bars[s]), ph, abort_flag, p.wait_polls);
 
         // ---- this pair's 16-token tiles of the page
         const uint32_t stg = (uint32_t)s * (uint32_t)U.bytes;   // byte offset of the stage
@@ -833,6 +863,8 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
                 const float fb = f16_bits_to_f32(*reinterpret_cast<const uint16_t*>(smem + kst + ksoff[0] + 8 * T::KS));
                 sc[0] *= fa; sc[1] *= fa; sc[2] *= fb; sc[3] *= fb;
             }
+            // q's power of two (and the K tensor scale) back into the fp32 scores
+            sc[0] *= hm0; sc[1] *= hm1; sc[2] *= hm0; sc[3] *= hm1;
             const bool oka = r < valid, okb = r + 8 < valid;
             if (!oka) sc[0] = sc[1] = -INFINITY;
             if (!okb) sc[2] = sc[3] = -INFINITY;
@@ -874,30 +906,55 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
             // product entirely (their P is 0, but 0 x NaN would still be NaN)
             const bool partial = valid < 16;
             uint32_t pb0 = 0, pb1 = 0;   // P'^T fragment (B operand)
+            // V scales folded into P': this lane's rows r and r + 8, one per
+            // chunk (INT8, MX) or one per row (FP8 row-256), rows past seq_len 0
+            constexpr int NVS = VFOLD ? (KV == RK_E4M3_ROW256 ? 1 : T::VC_HALF) : 1;
+            float vfa[NVS], vfb[NVS];
+            if constexpr (VFOLD) {
+                float smax = 0.f;
+#pragma unroll
+                for (int c = 0; c < NVS; c++) {
+                    if constexpr (KV == RK_E4M3_MX32) {
+                        vfa[c] = ue8m0_to_f32(smem[vst + vsoff[c]]);
+                        vfb[c] = ue8m0_to_f32(smem[vst + vsoff[c] + 8 * T::VS]);
+                    } else {
+                        vfa[c] = f16_bits_to_f32(*reinterpret_cast<const uint16_t*>(smem + vst + vsoff[c]));
+                        vfb[c] = f16_bits_to_f32(*reinterpret_cast<const uint16_t*>(smem + vst + vsoff[c] + 8 * T::VS));
+                    }
+                    vfa[c] = oka ? vfa[c] : 0.f;
+                    vfb[c] = okb ? vfb[c] : 0.f;
+                    smax = fmaxf(smax, fmaxf(vfa[c], vfb[c]));
+                }
+                if (__any_sync(0xffffffffu, smax > vthr)) {
+                    // raise the reference to the warp's largest scale (an exact power of two)
+                    const int en = exp2_floor(__uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(smax))));
+                    const float f = vthr > 0.f ? pow2i(ve - en) : 1.f;
+#pragma unroll
+                    for (int u = 0; u < T::DTILES / 2; u++) {
+                        o[u][0] *= f; o[u][1] *= f; o[u][2] *= f; o[u][3] *= f;
+                    }
+                    ve = en;
+                    vmul = pow2i(-en);
+                    vthr = pow2i(en + 4);
+                }
+#pragma unroll
+                for (int c = 0; c < NVS; c++) {
+                    vfa[c] *= vmul;
+                    vfb[c] *= vmul;
+                }
+            }
             if constexpr (KV == RK_E4M3_ROW256) {
-                const float fa = oka ? f16_bits_to_f32(*reinterpret_cast<const uint16_t*>(smem + vst + vsoff[0])) : 0.f;
-                const float fb = okb ? f16_bits_to_f32(*reinterpret_cast<const uint16_t*>(smem + vst + vsoff[0] + 8 * T::VS)) : 0.f;
-                pb0 = movtrans(pack_f16(p0 * fa, p1 * fa));
-                pb1 = movtrans(pack_f16(p2 * fb, p3 * fb));
-            } else if constexpr (KV != RK_INT8_G64 && KV != RK_E4M3_MX32) {
+                pb0 = movtrans(pack_f16(p0 * vfa[0], p1 * vfa[0]));
+                pb1 = movtrans(pack_f16(p2 * vfb[0], p3 * vfb[0]));
+            } else if constexpr (!VFOLD) {
                 pb0 = movtrans(pack_f16(p0, p1));
                 pb1 = movtrans(pack_f16(p2, p3));
             }
 #pragma unroll
             for (int cl = 0; cl < T::VC_HALF; cl++) {
                 if constexpr (KV == RK_INT8_G64 || KV == RK_E4M3_MX32) {
-                    float fa, fb;
-                    if constexpr (KV == RK_INT8_G64) {
-                        fa = f16_bits_to_f32(*reinterpret_cast<const uint16_t*>(smem + vst + vsoff[cl]));
-                        fb = f16_bits_to_f32(*reinterpret_cast<const uint16_t*>(smem + vst + vsoff[cl] + 8 * T::VS));
-                    } else {
-                        fa = ue8m0_to_f32(smem[vst + vsoff[cl]]);
-                        fb = ue8m0_to_f32(smem[vst + vsoff[cl] + 8 * T::VS]);
-                    }
-                    fa = oka ? fa : 0.f;
-                    fb = okb ? fb : 0.f;
-                    pb0 = movtrans(pack_f16(p0 * fa, p1 * fa));
-                    pb1 = movtrans(pack_f16(p2 * fb, p3 * fb));
+                    pb0 = movtrans(pack_f16(p0 * vfa[cl], p1 * vfa[cl]));
+                    pb1 = movtrans(pack_f16(p2 * vfb[cl], p3 * vfb[cl]));
                 }
                 uint32_t xa[2 * T::VCH], xb[2 * T::VCH];
                 slice_f16<KV, T::VNB, T::VCH>(lds_bytes<T::VNB>(smem + vt, voff[cl]), xa);
@@ -965,8 +1022,10 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
                 M0 = fmaxf(M0, wml[w * 16 + 2 * j]);
                 M1 = fmaxf(M1, wml[w * 16 + 2 * j + 1]);
             }
-            const float f0 = (m0 == -INFINITY) ? 0.f : exp2f(m0 - M0);
-            const float f1 = (m1 == -INFINITY) ? 0.f : exp2f(m1 - M1);
+            // this warp's outputs back in real units: o is held in units of 2^ve
+            const float vu = VFOLD ? pow2i(ve) : 1.f;
+            const float f0 = (m0 == -INFINITY) ? 0.f : exp2f(m0 - M0) * vu;
+            const float f1 = (m1 == -INFINITY) ? 0.f : exp2f(m1 - M1) * vu;
             if (tid < 8) {
                 float M = -INFINITY, Ls = 0.f;
                 for (int w = 0; w < 4; w++) M = fmaxf(M, wml[w * 16 + tid]);
@@ -1113,7 +1172,7 @@ static size_t fixed_smem(int D, int B, int pid_cap, int qs) {
     const size_t ostr = (size_t)D + 4;   // kOsmStride
     const size_t osm = 8 * ostr * 4 > 8192 ? 8 * ostr * 4 : 8192;
     const size_t qst = 8 * (size_t)D * 2 * qs;
-    return 8 * kMaxStages + 4 * kMaxStages + 32 + osm + qst + 4 * 16 * 4 + 16 * 4 + 16 + 4 * (size_t)(B + 1) +
+    return 8 * kMaxStages + 4 * kMaxStages + 32 + osm + qst + 4 * 16 * 4 + 16 * 4 + 8 * 4 + 16 + 4 * (size_t)(B + 1) +
            4 * (size_t)pid_cap + 128;
 }
 

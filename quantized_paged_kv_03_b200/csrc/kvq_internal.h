@@ -67,9 +67,11 @@ struct DecodeParams {
     int B;
     void* out;
     int out_fp32;
-    float q_mult;                // softmax_scale * log2(e) * K tensor scale
+    float q_mult;                // softmax_scale * log2(e)
+    float k_tmult;               // K tensor scale (FP8_TENSOR; 1 otherwise), applied to fp32 scores
     float o_mult;                // V tensor scale (1 otherwise)
     bool rot_k, rot_v;
+    long wait_polls;             // polls of a pipeline wait before it gives up
     float* partials;             // [gridDim.x][2][16 + 8 * D]: (max, sum, output) of cut segments
     unsigned* barrier;           // grid barrier: [0] arrivals (zero between calls), [1] generation
     uint32_t* status;
@@ -78,7 +80,12 @@ struct DecodeParams {
     const uint16_t* k_new;       // fused append: bf16 [B][H][D] rows of each sequence's newest
     const uint16_t* v_new;       //   token (position seq_len - 1), or null for decode only
     float k_scale, v_scale;      // per-tensor scales of the append (FP8_TENSOR)
+    int max_seq_len;             // host-side: sizes the plan
 };
+
+// Polls a pipeline wait makes before it gives up (the default unless a test
+// changed it with kvq_debug_set_wait_polls).
+long wait_polls();
 
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
 cudaError_t launch_read_rows(const ReadParams& p, cudaStream_t s);
@@ -101,5 +108,19 @@ bool decode_supported(int fmt, int D);
 }  // namespace kvq
 
 struct kvq_cache;
+
+namespace kvq {
+// The C-ABI layer's decode path in steps (kvq_api.cu), shared by every decode
+// entry point: validate on the host (kvq_status codes; *batch0 set when batch
+// is 0 and there is nothing to launch), plan for the current device, launch
+// on a workspace.
+int decode_setup(kvq_cache* cache, int32_t layer, const void* k_new, const void* v_new, const void* q,
+                 int32_t n_q_heads, const int32_t* block_table, int32_t max_pages_per_seq, const int32_t* seq_lens,
+                 int32_t batch, int32_t max_seq_len, void* out, int32_t out_fp32, float softmax_scale,
+                 DecodeParams* p, bool* batch0);
+int decode_plan(DecodeParams* p, DecodePlan* plan);
+int decode_launch(DecodeParams* p, const DecodePlan& plan, void* workspace, cudaStream_t stream);
+}  // namespace kvq
+
 // Page layout of a cache handle (defined with the handle in kvq_api.cu).
 const kvq::Layout* kvq_cache_layout(const kvq_cache* cache);

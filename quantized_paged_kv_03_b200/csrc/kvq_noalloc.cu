@@ -48,26 +48,25 @@ extern "C" int kvq_decode_attention_noalloc(kvq_cache* cache, int32_t layer, con
                                             const int32_t* block_table, int32_t max_pages_per_seq,
                                             const int32_t* seq_lens, int32_t batch, int32_t max_seq_len,
                                             void* out, int32_t out_fp32, float softmax_scale, void* stream) {
-    if (!cache) return KVQ_ERR_ARG;
-    if (batch == 0) return KVQ_OK;
-    const size_t need = kvq_decode_workspace_bytes(cache, batch, n_q_heads, max_seq_len);
-    if (need == 0) return KVQ_ERR_SHAPE;
+    // the same validation as kvq_decode_attention (same status codes), then the
+    // scratch size limit, then -- only for a call that will launch -- the memset
+    kvq::DecodeParams p;
+    kvq::DecodePlan plan;
+    bool none = false;
+    int st = kvq::decode_setup(cache, layer, nullptr, nullptr, q, n_q_heads, block_table, max_pages_per_seq,
+                               seq_lens, batch, max_seq_len, out, out_fp32, softmax_scale, &p, &none);
+    if (st != KVQ_OK || none) return st;
+    if ((st = kvq::decode_plan(&p, &plan)) != KVQ_OK) return st;
+    const size_t need = kvq::decode_workspace_bytes(p.L, batch, p.HB, plan.grid);
     if (need > (size_t)KVQ_NOALLOC_SCRATCH_BYTES) return KVQ_ERR_WORKSPACE;
     void* scratch = nullptr;
-    int st = scratch_for_current_device(&scratch);
+    st = scratch_for_current_device(&scratch);
     if (st != KVQ_OK) return st;
     // The array keeps whatever the previous call left there: clear the part
     // the kernel expects to start at zero.
-    const kvq::Layout* L = kvq_cache_layout(cache);
-    const int G = n_q_heads / L->H, HB = (G + 7) / 8;
-    kvq::DecodePlan plan;
-    if (kvq::plan_decode(*L, batch, HB, max_seq_len, &plan) != cudaSuccess) return KVQ_ERR_CUDA;
     size_t zoff = 0, zbytes = 0;
-    kvq::decode_workspace_zero_region(*L, batch, HB, plan.grid, &zoff, &zbytes);
-    if (zoff + zbytes > (size_t)KVQ_NOALLOC_SCRATCH_BYTES) return KVQ_ERR_WORKSPACE;
+    kvq::decode_workspace_zero_region(p.L, batch, p.HB, plan.grid, &zoff, &zbytes);
     if (cudaMemsetAsync((unsigned char*)scratch + zoff, 0, zbytes, (cudaStream_t)stream) != cudaSuccess)
         return KVQ_ERR_CUDA;
-    return kvq_decode_attention(cache, layer, q, n_q_heads, block_table, max_pages_per_seq, seq_lens, batch,
-                                max_seq_len, out, out_fp32, softmax_scale, scratch, KVQ_NOALLOC_SCRATCH_BYTES,
-                                stream);
+    return kvq::decode_launch(&p, plan, scratch, (cudaStream_t)stream);
 }

@@ -40,12 +40,16 @@
 //    epilogue (the matrix is symmetric and its own inverse).
 //
 // Precision: q and the key/value tiles are fp16 (bf16 for BF16 keys).  Codes
-// of every format are exact in fp16; a dequantised value code x scale is exact
-// for E2M1 x UE4M3, E4M3 per tensor (the tensor scale is applied in fp32) and
-// MX E4M3 x 2^k in fp16's normal range, and rounded once (nearest-even,
-// relative 2^-11) for INT8 and E4M3 row-256 with their fp16 scales.  Stored
-// values beyond fp16's range (|x| > 65504) saturate; the decode kernel, which
-// applies scales in fp32, has no such limit.
+// of every format are exact in fp16.  For INT8, E4M3 row-256 and MX, whose
+// scales span more than fp16's range, a tile's values enter as
+// code x scale x 2^-e, e the exponent of the tile's largest scale; the 2^e goes
+// back in fp32 (keys: into the score multiplier; values: into P, against a
+// running reference exponent of the block, with O rescaled when it rises).  So
+// values neither saturate nor lose precision to fp16 subnormals whatever their
+// magnitude; what remains is one nearest-even rounding (relative 2^-11) of
+// code x scale for INT8 and E4M3 row-256, whose fp16 scales carry 11 bits.
+// E2M1 x UE4M3 and per-tensor E4M3 (tensor scales applied in fp32) are exact.
+// q itself goes to fp16 as given: |q| up to 65504, full precision above 2^-14.
 #include "kvq_prefill.h"
 #include "kvq_tc.cuh"
 
@@ -77,8 +81,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t phase) {
 // Bounded wait: gives up after kPrefillWaitPolls polls, or at once when another
 // thread already gave up (`abort` set), so a copy that never lands cannot hang
 // the CTA; the caller records the timeout in the status word.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t phase, volatile int* abort) {
-    for (long i = 0; i < kPrefillWaitPolls; i++) {
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t phase, volatile int* abort,
+                                          long polls = kPrefillWaitPolls) {
+    for (long i = 0; i < polls; i++) {
         if (mbar_try_wait(bar, phase)) return true;
         if (*abort) return false;
     }
@@ -138,8 +143,12 @@ __device__ __forceinline__ uint32_t p_off(int r, int c) { return (uint32_t)((c >
 
 // Dequantise one 16-byte code chunk (chunk j of row t, logical order) into the
 // tile, with the row's scales applied: 8, 16 or 32 elements by the code width.
+// `smul` = 2^-e, e the tile's scale exponent (tile_scale_exp): INT8, E4M3
+// row-256 and MX scales enter as scale x 2^-e, so every dequantised value of
+// the tile lies below 2 x the largest code, inside fp16's range.
 template <int KIND, int D>
-__device__ __forceinline__ void dequant_chunk(const uint4 w, const uint8_t* srow, int j, uint8_t* tile, int t, int T) {
+__device__ __forceinline__ void dequant_chunk(const uint4 w, const uint8_t* srow, int j, uint8_t* tile, int t, int T,
+                                              float smul) {
     constexpr int SB = kind_scale_bytes(KIND);
     const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
     if constexpr (kind_bits(KIND) == 16) {
@@ -169,12 +178,13 @@ __device__ __forceinline__ void dequant_chunk(const uint4 w, const uint8_t* srow
         if constexpr (KIND == RK_INT8_G64 || KIND == RK_E4M3_ROW256) {
             // fp16 scale: one nearest-even rounding of code x scale
             const int g = j * 16 / kind_group(KIND);
-            const uint32_t sc = splat16((uint32_t)srow[SB * g] | ((uint32_t)srow[SB * g + 1] << 8));
+            const float sf = f16_bits_to_f32((uint32_t)srow[SB * g] | ((uint32_t)srow[SB * g + 1] << 8)) * smul;
+            const uint32_t sc = splat16(__half_as_ushort(__float2half_rn(sf)));
 #pragma unroll
             for (int i = 0; i < 8; i++) h[i] = mul_f16x2(h[i], sc);
         } else if constexpr (KIND == RK_E4M3_MX32) {
             // UE8M0 scale 2^(e-127): applied in fp32 (exact), then to fp16
-            const float sc = ue8m0_to_f32(srow[j * 16 / 32]);
+            const float sc = ue8m0_to_f32(srow[j * 16 / 32]) * smul;
 #pragma unroll
             for (int i = 0; i < 8; i++) {
                 const float2 f = f16x2_to_f32(h[i]);
@@ -196,7 +206,7 @@ __device__ __forceinline__ void dequant_chunk(const uint4 w, const uint8_t* srow
 // that a masked key's weight 0 never meets a non-finite value.
 template <int KIND, int D>
 __device__ __forceinline__ void dequant_tile(const uint8_t* codes, const uint8_t* scales, uint8_t* tile, int T,
-                                             int lgT, int valid, int tid) {
+                                             int lgT, int valid, int tid, float smul) {
     constexpr int CB = row_code_bytes(KIND, D), SB = row_scale_bytes(KIND, D);
     constexpr int CPR = CB / 16;                       // chunks per row (a power of two)
     constexpr int EPC = 128 / kind_bits(KIND);         // elements per chunk
@@ -221,9 +231,41 @@ __device__ __forceinline__ void dequant_tile(const uint8_t* codes, const uint8_t
             for (int e = 0; e < EPC / 8; e++)
                 *reinterpret_cast<uint4*>(tile + kv_off(t, j * EPC + 8 * e, T)) = make_uint4(0, 0, 0, 0);
         } else {
-            dequant_chunk<KIND, D>(w[i], scales + t * SB, j, tile, t, T);
+            dequant_chunk<KIND, D>(w[i], scales + t * SB, j, tile, t, T, smul);
         }
     }
+}
+
+// Kinds whose dequantised values are normalised per tile (fp16 or UE8M0
+// scales, whose range exceeds fp16's); E2M1 x UE4M3, per-tensor E4M3 and the
+// 16-bit kinds are exact in fp16 as they are.
+__host__ __device__ constexpr bool scale_normalised(int k) {
+    return k == RK_INT8_G64 || k == RK_E4M3_ROW256 || k == RK_E4M3_MX32;
+}
+
+// floor(log2) of the largest scale among the first `rows` scale rows of a stage
+// (rows of SB bytes, the rows that hold tokens of the sequence: later rows may
+// hold stale bytes), the same in every lane: each warp reads the rows itself,
+// so no CTA barrier is needed.  0 when every scale is zero.
+template <int KIND, int D>
+__device__ __forceinline__ int tile_scale_exp(const uint8_t* scales, int rows, int lane) {
+    constexpr int SB = row_scale_bytes(KIND, D);
+    const int nb = rows * SB;
+    uint32_t mx = 0;
+    for (int i = lane; 4 * i < nb; i += 32) {
+        const int rem = nb - 4 * i;
+        const uint32_t keep = rem >= 4 ? 0xFFFFFFFFu : (1u << (8 * rem)) - 1u;
+        const uint32_t w = reinterpret_cast<const uint32_t*>(scales)[i] & keep;
+        if constexpr (KIND == RK_E4M3_MX32) {
+            mx = max(mx, max(max(w & 0xFFu, (w >> 8) & 0xFFu), max((w >> 16) & 0xFFu, w >> 24)));
+        } else {
+            mx = max(mx, max(w & 0x7FFFu, (w >> 16) & 0x7FFFu));
+        }
+    }
+    mx = __reduce_max_sync(0xffffffffu, mx);
+    if (mx == 0) return 0;
+    if constexpr (KIND == RK_E4M3_MX32) return (int)mx - 127;
+    else return (int)max(mx >> 10, 1u) - 15;   // fp16 exponent field (subnormals: 2^-14)
 }
 
 // Stage the block's 128 query rows into sQ: row r is global row R0 + r of the
@@ -231,8 +273,8 @@ __device__ __forceinline__ void dequant_tile(const uint8_t* codes, const uint8_t
 // (rotated by the Hadamard-256 first when K is rotated), or the bf16 bits
 // themselves for BF16 keys; rows past the chunk are zeros.  One warp per row.
 template <int D, bool QBF16>
-__device__ __forceinline__ void stage_q(const PrefillParams& p, uint8_t* sQ, int64_t qrow0, int hh, int64_t R0,
-                                        int64_t rows_total, int warp, int lane) {
+__device__ __forceinline__ void stage_q(const PrefillParams& p, uint8_t* sQ, float* qrm, int64_t qrow0, int hh,
+                                        int64_t R0, int64_t rows_total, int warp, int lane) {
     constexpr int EPL = D / 32;
     for (int r = warp; r < kPrefillRows; r += kPrefillThreads / 32) {
         const int64_t gr = R0 + r;
@@ -251,6 +293,7 @@ __device__ __forceinline__ void stage_q(const PrefillParams& p, uint8_t* sQ, int
             }
         }
         uint32_t h[EPL / 2];
+        float rm = 1.f;   // the row's power of two, returned to its scores in fp32
         if constexpr (QBF16) {
 #pragma unroll
             for (int i = 0; i < EPL / 2; i++) h[i] = bits[i];
@@ -264,9 +307,19 @@ __device__ __forceinline__ void stage_q(const PrefillParams& p, uint8_t* sQ, int
             if constexpr (D == 256) {
                 if (p.rot_k) fwht256_warp(x, lane);
             }
+            // normalised so that the row's largest element lies in [1, 2): fp16
+            // keeps full precision whatever q's magnitude
+            float amax = 0.f;
 #pragma unroll
-            for (int i = 0; i < EPL / 2; i++) h[i] = enc_f16x2_sat(x[2 * i], x[2 * i + 1]);
+            for (int i = 0; i < EPL; i++) amax = fmaxf(amax, fabsf(x[i]));
+            amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(amax)));
+            const int eq = amax > 0.f ? exp2_floor(amax) : 0;
+            const float nq = pow2i(-eq);
+            rm = pow2i(eq);
+#pragma unroll
+            for (int i = 0; i < EPL / 2; i++) h[i] = enc_f16x2_sat(x[2 * i] * nq, x[2 * i + 1] * nq);
         }
+        if (lane == 0) qrm[r] = rm;
         if constexpr (EPL == 8) {
             *reinterpret_cast<uint4*>(sQ + tc::blk(r, lane * 8, D)) = make_uint4(h[0], h[1], h[2], h[3]);
         } else {
@@ -293,7 +346,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const Prefi
     uint8_t* ring = smem + prefill_region0(D, T);
     uint64_t* bars = reinterpret_cast<uint64_t*>(ring + (size_t)p.stages * p.st_bytes);
     float* red = reinterpret_cast<float*>(bars + p.stages + 2);   // [2][128]: per-half row values
-    uint32_t* tslot = reinterpret_cast<uint32_t*>(red + 2 * kPrefillRows);
+    float* qrm = red + 2 * kPrefillRows;                          // [128]: each row's q power of two
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(qrm + kPrefillRows);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -331,7 +385,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const Prefi
 
     // key tile k of this sequence into stage s: the whole page slab in one copy
     // when the tile is the page, else the tile's rows of the slab's four arrays
+    // thread 0's counts of what it handed to the copy engine and the tensor
+    // core: copies issued (ring positions 0 .. n_issued - 1), S and O commits
+    uint32_t n_issued = 0, n_s = 0, n_o = 0;
     auto issue = [&](uint32_t seq, int k) {
+        if (*abort_flag) return;   // after a wait gave up nothing new is started
+        n_issued = seq + 1;
         const int s = (int)(seq % (uint32_t)p.stages);
         const int t0 = k * T;
         const int page = t0 / p.L.P;   // past the block table's width: a sequence longer than it holds
@@ -358,7 +417,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const Prefi
         }
     };
     auto wait_or_flag = [&](uint32_t bar, uint32_t phase) {
-        if (!mbar_wait(bar, phase, abort_flag) && lane == 0) atomicOr(p.status, kStatusWaitTimeout);
+        if (!mbar_wait(bar, phase, abort_flag, p.wait_polls) && lane == 0) atomicOr(p.status, kStatusWaitTimeout);
     };
 
     uint32_t seq = 0;   // key tiles consumed by this CTA: ring stage seq % stages, phase seq / stages
@@ -370,7 +429,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const Prefi
         const int ntiles = pos_hi >= 0 ? pos_hi / T + 1 : 0;
         if (tid == 0)
             for (int k = 0; k < p.stages && k < ntiles; k++) issue(seq + k, k);
-        stage_q<D, KBF>(p, sQ, qrow0, hh, R0, rows_total, warp, lane);
+        stage_q<D, KBF>(p, sQ, qrm, qrow0, hh, R0, rows_total, warp, lane);
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 
         // this thread's row position (-1: past the chunk, no keys) and the
@@ -380,7 +439,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const Prefi
         const int64_t gfirst = R0 + g4 * 32;
         const int gpos_min = gfirst + 31 < rows_total ? Ls - n + (int)(gfirst / p.G) : -1;
         float m_ref = -INFINITY, l_part = 0.f;
+        // value tiles enter scaled by 2^-eV (their own scale exponent); P carries
+        // 2^(eV - ev_ref) so that O stays in units of 2^ev_ref, a reference raised
+        // (O rescaled) when a tile's exponent exceeds it by more than 4
+        int ev_ref = 0;
+        bool ev_set = false;
         __syncthreads();   // q staged
+        const float qrow = qrm[r];
 
         for (int k = 0; k < ntiles; k++, seq++, rnd++) {
             const int s = (int)(seq % (uint32_t)p.stages);
@@ -388,24 +453,45 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const Prefi
             wait_or_flag(smem_addr(&bars[s]), (seq / (uint32_t)p.stages) & 1u);
             const int t0 = k * T;
             const int valid = min(T, Ls - t0);
+            // the tile's scale exponents (every warp computes them from the stage)
+            int ek = 0, evt = 0;
+            if constexpr (scale_normalised(KK)) ek = tile_scale_exp<KK, D>(st + p.st_ks, valid, lane);
+            if constexpr (scale_normalised(KV)) evt = tile_scale_exp<KV, D>(st + p.st_vs, valid, lane);
             // keys first: S of this tile can start while the values are dequantised
-            dequant_tile<KK, D>(st, st + p.st_ks, sK, T, lgT, valid, tid);
+            dequant_tile<KK, D>(st, st + p.st_ks, sK, T, lgT, valid, tid, pow2i(-ek));
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncthreads();
-            if (tid == 0) {
+            if (tid == 0 && !*abort_flag) {
                 tc::fence_after();
 #pragma unroll
                 for (int kk = 0; kk < D / 16; kk++)
                     tc::mma_f16(tS, tc::sdesc(aQ + 256 * kk, 128, 16 * D), tc::sdesc(aK + kk * 32 * T, 16 * T, 128),
                                 idS, kk > 0);
                 tc::commit(barS);
+                n_s++;
             }
             if (k > 0) {   // the previous P V still reads the value and P tiles
                 wait_or_flag(barO, (rnd - 1) & 1u);
                 tc::fence_after();
             }
-            dequant_tile<KV, D>(st + p.st_vc, st + p.st_vs, sV, T, lgT, valid, tid);
+            dequant_tile<KV, D>(st + p.st_vc, st + p.st_vs, sV, T, lgT, valid, tid, pow2i(-evt));
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            // the value reference: set by the first tile, raised when this tile's
+            // exponent is more than 2^4 above it (the same decision in every thread)
+            float vcorr = 1.f;
+            bool vresc = false;
+            if constexpr (scale_normalised(KV)) {
+                if (!ev_set || evt > ev_ref + 4) {
+                    if (ev_set) {
+                        vcorr = pow2i(ev_ref - evt);
+                        vresc = true;
+                    }
+                    ev_ref = evt;
+                    ev_set = true;
+                }
+            }
+            const int dv = evt - ev_ref;   // <= 4: P of this tile carries 2^dv
+            const float qm = p.q_mult * pow2i(ek) * qrow;
 
             // ---- scores of this thread's row, columns [32 h, 32 h + 32) of the tile
             wait_or_flag(barS, rnd & 1u);
@@ -421,7 +507,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const Prefi
                 const bool mask = t0 + T - 1 > gpos_min;
 #pragma unroll
                 for (int i = 0; i < 32; i++) {
-                    float x = __uint_as_float(v[i]) * p.q_mult;
+                    float x = __uint_as_float(v[i]) * qm;
                     if (c0 + i >= T || (mask && t0 + c0 + i > pos)) x = -INFINITY;
                     sv[i] = x;
                     mx = fmaxf(mx, x);
@@ -440,7 +526,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const Prefi
                 corr = ex2(m_ref - mt);
                 m_ref = mt;
             }
-            const float base = m_ref == -INFINITY ? 0.f : m_ref;
+            // P of this tile = 2^(s - m_ref + dv): the value tile's 2^dv is folded in
+            const float base = (m_ref == -INFINITY ? 0.f : m_ref) - (float)dv;
             float rs = 0.f;
             if (active) {
 #pragma unroll
@@ -456,9 +543,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const Prefi
                         *reinterpret_cast<uint4*>(sP + p_off(r, c0 + 8 * q8)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
                 }
             }
-            l_part = l_part * corr + rs;
-            if (k > 0 && __any_sync(0xffffffffu, resc)) {
+            l_part = l_part * corr + rs * pow2i(-dv);
+            if (k > 0 && (vresc || __any_sync(0xffffffffu, resc))) {
                 // O of this thread's row, columns [h D/2, h D/2 + D/2), times corr
+                corr *= vcorr;
 #pragma unroll 1
                 for (int cc = 0; cc < D / 2; cc += 32) {
                     uint32_t v[32];
@@ -474,7 +562,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const Prefi
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             tc::fence_before();
             __syncthreads();   // P and the value tile written, O rescaled
-            if (tid == 0) {
+            if (tid == 0 && !*abort_flag) {
                 tc::fence_after();
 #pragma unroll
                 for (int kk = 0; kk < kMaxT / 16; kk++)
@@ -482,6 +570,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const Prefi
                         tc::mma_f16(tO, tc::sdesc(aP + kk * 2 * (kPrefillRows * 16), kPrefillRows * 16, 128),
                                     tc::sdesc(aV + 256 * kk, 128, 16 * T), idO, k > 0 || kk > 0);
                 tc::commit(barO);
+                n_o++;
             }
         }
 
@@ -493,7 +582,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const Prefi
         red[h * kPrefillRows + r] = l_part;
         __syncthreads();
         const float l = red[r] + red[kPrefillRows + r];
-        const float inv = l > 0.f ? p.o_mult / l : 0.f;
+        const float inv = l > 0.f ? p.o_mult / l * pow2i(ev_ref) : 0.f;   // O is in units of 2^ev_ref
         float* so = sO + r * OST + h * (D / 2);
 #pragma unroll 1
         for (int cc = 0; cc < D / 2; cc += 32) {
@@ -542,6 +631,17 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const Prefi
             }
         }
         __syncthreads();   // the shared region is free for the next block
+    }
+    if (tid == 0 && *abort_flag) {
+        // a wait gave up: before the tensor memory is freed and the CTA exits,
+        // wait (with the default bound) for what was already handed out -- the
+        // last copy into each ring stage, and the last S and O products (each
+        // is issued only after the previous one of its kind was waited for)
+        int ignore = 0;
+        for (uint32_t j = n_issued > (uint32_t)p.stages ? n_issued - p.stages : 0; j < n_issued; j++)
+            (void)mbar_wait(smem_addr(&bars[j % p.stages]), (j / p.stages) & 1u, &ignore);
+        if (n_s) (void)mbar_wait(barS, (n_s - 1) & 1u, &ignore);
+        if (n_o) (void)mbar_wait(barO, (n_o - 1) & 1u, &ignore);
     }
     tc::fence_before();
     __syncthreads();

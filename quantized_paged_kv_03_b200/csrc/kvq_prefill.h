@@ -19,9 +19,9 @@ KVQ_HD constexpr int64_t prefill_region0(int D, int T) {
     return ((ops > osm ? ops : osm) + 1023) & ~int64_t(1023);
 }
 // Bytes after the stage ring: the ring's mbarriers, the S and O completion
-// mbarriers, the row exchange buffer (2 x 128 floats), the tensor-memory
-// address and the abort flag.
-KVQ_HD constexpr int64_t prefill_tail_bytes(int stages) { return 8 * (stages + 2) + 2 * kPrefillRows * 4 + 16; }
+// mbarriers, the row exchange buffer (2 x 128 floats), the rows' q multipliers
+// (128 floats), the tensor-memory address and the abort flag.
+KVQ_HD constexpr int64_t prefill_tail_bytes(int stages) { return 8 * (stages + 2) + 3 * kPrefillRows * 4 + 16; }
 
 struct PrefillParams {
     Layout L;
@@ -38,6 +38,7 @@ struct PrefillParams {
     float q_mult;                // softmax_scale * log2(e) * K tensor scale
     float o_mult;                // V tensor scale (1 otherwise)
     bool rot_k, rot_v;
+    long wait_polls;             // polls of a pipeline wait before it gives up
     uint32_t* status;
     // set by the launch from the plan
     int T;                       // key tile: tokens per stage (divides the page size)

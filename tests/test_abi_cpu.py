@@ -33,7 +33,7 @@ def test_library_exports_every_declared_symbol(L):
     for n in names:
         assert hasattr(L, n), n
     assert sorted(K.exported_symbols()) == names
-    assert L.kvq_version() == 2
+    assert L.kvq_version() == 3
 
 
 def test_token_bytes_table(L):
@@ -126,6 +126,43 @@ def test_calls_reject_bad_arguments_before_launch(L):
     assert L.kvq_dequant(h, 3, p, 3, p, p, None) == 1
     assert L.kvq_status_string(4) == b"pool or workspace too small"
     L.kvq_cache_destroy(h)
+
+
+def test_noalloc_decode_rejects_what_decode_rejects(L):
+    """The allocation-free entry point validates through the same host checks
+    as kvq_decode_attention and returns the same status codes, before any CUDA
+    call (this runs without a GPU)."""
+    h = ctypes.c_void_p()
+    fake = ctypes.c_void_p(1 << 20)
+    d = _desc(H=2)
+    assert L.kvq_cache_create(ctypes.byref(d), fake, L.kvq_cache_bytes(ctypes.byref(d)), ctypes.byref(h)) == 0
+    p = ctypes.c_void_p(1 << 21)
+    odd = ctypes.c_void_p((1 << 21) + 8)
+    #   (layer, q, n_q_heads, max_pages, batch, max_seq_len, out, scale) -> status
+    cases = [((1, p, 4, 4, 2, 256, p, 0.0), 1),      # layer out of range
+             ((0, p, 5, 4, 2, 256, p, 0.0), 3),      # heads not a multiple of kv-heads
+             ((0, p, 0, 4, 2, 256, p, 0.0), 1),      # no query heads
+             ((0, p, 4, 4, -1, 256, p, 0.0), 1),     # negative batch
+             ((0, p, 4, 4, 5000, 256, p, 0.0), 3),   # batch beyond the limit
+             ((0, p, 4, 2, 2, 256, p, 0.0), 3),      # max_seq_len beyond the block table
+             ((0, odd, 4, 4, 2, 256, p, 0.0), 1),    # misaligned q
+             ((0, p, 4, 4, 2, 256, odd, 0.0), 1),    # misaligned out
+             ((0, None, 4, 4, 2, 256, p, 0.0), 1),   # null q
+             ((0, p, 4, 4, 2, 256, p, -1.0), 1),     # negative scale
+             ((0, p, 4, 4, 0, 256, p, 0.0), 0)]      # batch 0: nothing to do
+    for (layer, q, hq, mp, B, ms, out, sc), want in cases:
+        a = L.kvq_decode_attention(h, layer, q, hq, p, mp, p, B, ms, out, 1, sc, p, 1 << 20, None)
+        b = L.kvq_decode_attention_noalloc(h, layer, q, hq, p, mp, p, B, ms, out, 1, sc, None)
+        assert a == b == want, (layer, hq, mp, B, ms, sc, a, b)
+    # a call that would launch without a workspace is an argument error
+    assert L.kvq_decode_attention(h, 0, p, 4, p, 4, p, 2, 256, p, 1, 0.0, None, 1 << 20, None) == 1
+    L.kvq_cache_destroy(h)
+
+
+def test_wait_limit_setting_round_trips(L):
+    prev = L.kvq_debug_set_wait_polls(7)
+    assert L.kvq_debug_set_wait_polls(-1) == 7       # negative restores the default
+    assert L.kvq_debug_set_wait_polls(-1) == prev == 1 << 22
 
 
 def test_python_binding_fails_loudly_without_library(monkeypatch, tmp_path):

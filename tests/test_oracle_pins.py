@@ -31,7 +31,7 @@ def test_token_bytes_match_the_pages_table():
     # "≈51% / ≈50% / ≈28% / ≈39%" of BF16 (the table truncates: 528/1024 = 51.6%)
     for name, pct in (("int8_g64", 51), ("fp8_row256", 50), ("nvfp4_g16", 28), ("k8v4", 39)):
         assert math.floor(100 * O.token_bytes(NAMES[name], D) / 1024) == pct
-    # "接近 3.5 倍": context at fixed memory grows by 1024 / 288
+    # the NVFP4 paragraph's capacity figure (about 3.5x): context at fixed memory grows by 1024 / 288
     r = O.token_bytes(O.BF16, D) / O.token_bytes(O.NVFP4_G16, D)
     assert 3.4 < r < 3.6
 

@@ -6,7 +6,8 @@ call cudaMalloc to provide a workspace.  This entry point keeps its scratch in
 a fixed array inside the library instead.  The test calls it through the C ABI
 twice in a row and checks both results against the workspace-taking
 kvq_decode_attention on the same inputs, within the attention tolerance used
-by the other decode tests.  This file is named to be collected last."""
+by the other decode tests -- and, since it is the same kernel on the same
+inputs, bit for bit.  This file is named to be collected last."""
 import ctypes
 
 import numpy as np
@@ -43,8 +44,9 @@ def test_noalloc_decode_matches_workspace_decode_twice():
                                             out.data_ptr(), 1, ctypes.c_float(0.0), stream)
         assert st == 0, L.kvq_status_string(st)
         torch.cuda.synchronize()
-        diff = np.abs(out.cpu().numpy().astype(np.float64) - ref.cpu().numpy().astype(np.float64))
-        assert (diff <= ATTN_TOL * vm).all()
+        got, want = out.cpu().numpy().astype(np.float64), ref.cpu().numpy().astype(np.float64)
+        assert (np.abs(got - want) <= ATTN_TOL * vm).all()
+        assert np.array_equal(got, want)
     assert c.read_device_status() == 0
 
 
