@@ -469,7 +469,7 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
     extern __shared__ __align__(128) uint8_t smem[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int r = lane >> 2, j = lane & 3;
-    const int tw = warp & 3, hf = warp >> 2;     // tile slot, head_dim half
+    const int tw = warp >> 1, hf = warp & 1;     // tile slot, head_dim half (the pair on two schedulers)
     const int H = p.L.H, P = p.L.P, HB = p.HB, HH = H * HB, B = p.B;
     const int64_t slab = p.L.slab;            // page slab stride in HBM
     const SpanLayout& U = p.U;                // what one stage holds

@@ -41,15 +41,18 @@
 //
 // Precision: q and the key/value tiles are fp16 (bf16 for BF16 keys).  Codes
 // of every format are exact in fp16.  For INT8, E4M3 row-256 and MX, whose
-// scales span more than fp16's range, a tile's values enter as
-// code x scale x 2^-e, e the exponent of the tile's largest scale; the 2^e goes
-// back in fp32 (keys: into the score multiplier; values: into P, against a
-// running reference exponent of the block, with O rescaled when it rises).  So
-// values neither saturate nor lose precision to fp16 subnormals whatever their
-// magnitude; what remains is one nearest-even rounding (relative 2^-11) of
-// code x scale for INT8 and E4M3 row-256, whose fp16 scales carry 11 bits.
-// E2M1 x UE4M3 and per-tensor E4M3 (tensor scales applied in fp32) are exact.
-// q itself goes to fp16 as given: |q| up to 65504, full precision above 2^-14.
+// scales span more than fp16's range, values enter as code x scale x 2^-e, e
+// the exponent of the sequence's largest K (or V) scale, found by one pass
+// over the scale rows when the CTA starts; the 2^e goes back in fp32 (keys:
+// into the score multiplier, values: into the output's normalisation).  So no
+// value saturates, and the largest ones keep full fp16 precision whatever
+// their magnitude; values far below the sequence's largest (by 2^14 or more)
+// lose precision to fp16 subnormals, an absolute error below 2^-25 of the
+// largest, negligible against the tolerance, which scales with max|V|.  What
+// remains is one nearest-even rounding (relative 2^-11) of code x scale for
+// INT8 and E4M3 row-256, whose fp16 scales carry 11 bits.  E2M1 x UE4M3 and
+// per-tensor E4M3 (tensor scales applied in fp32) are exact.  q is normalised
+// per row by a power of two (returned in fp32), so its magnitude is free too.
 #include "kvq_prefill.h"
 #include "kvq_tc.cuh"
 
@@ -143,9 +146,9 @@ __device__ __forceinline__ uint32_t p_off(int r, int c) { return (uint32_t)((c >
 
 // Dequantise one 16-byte code chunk (chunk j of row t, logical order) into the
 // tile, with the row's scales applied: 8, 16 or 32 elements by the code width.
-// `smul` = 2^-e, e the tile's scale exponent (tile_scale_exp): INT8, E4M3
-// row-256 and MX scales enter as scale x 2^-e, so every dequantised value of
-// the tile lies below 2 x the largest code, inside fp16's range.
+// `smul` = 2^-e, e the sequence's scale exponent (sequence_scale_exps): INT8,
+// E4M3 row-256 and MX scales enter as scale x 2^-e, so every dequantised value
+// lies below 2 x the largest code, inside fp16's range.
 template <int KIND, int D>
 __device__ __forceinline__ void dequant_chunk(const uint4 w, const uint8_t* srow, int j, uint8_t* tile, int t, int T,
                                               float smul) {
@@ -243,29 +246,80 @@ __host__ __device__ constexpr bool scale_normalised(int k) {
     return k == RK_INT8_G64 || k == RK_E4M3_ROW256 || k == RK_E4M3_MX32;
 }
 
-// floor(log2) of the largest scale among the first `rows` scale rows of a stage
-// (rows of SB bytes, the rows that hold tokens of the sequence: later rows may
-// hold stale bytes), the same in every lane: each warp reads the rows itself,
-// so no CTA barrier is needed.  0 when every scale is zero.
-template <int KIND, int D>
-__device__ __forceinline__ int tile_scale_exp(const uint8_t* scales, int rows, int lane) {
-    constexpr int SB = row_scale_bytes(KIND, D);
-    const int nb = rows * SB;
+// Largest scale magnitude (as comparable bits: the fp16 pattern without its
+// sign, or the UE8M0 byte) among `nb` bytes of scale rows at `src`, which
+// is 16-byte aligned; bytes past nb are ignored.  Pieces of 16 bytes, lane l
+// taking pieces l, l + 32, ...
+template <int KIND>
+__device__ __forceinline__ uint32_t scale_bits_max(const uint8_t* src, int nb, int lane) {
     uint32_t mx = 0;
-    for (int i = lane; 4 * i < nb; i += 32) {
-        const int rem = nb - 4 * i;
-        const uint32_t keep = rem >= 4 ? 0xFFFFFFFFu : (1u << (8 * rem)) - 1u;
-        const uint32_t w = reinterpret_cast<const uint32_t*>(scales)[i] & keep;
-        if constexpr (KIND == RK_E4M3_MX32) {
-            mx = max(mx, max(max(w & 0xFFu, (w >> 8) & 0xFFu), max((w >> 16) & 0xFFu, w >> 24)));
-        } else {
-            mx = max(mx, max(w & 0x7FFFu, (w >> 16) & 0x7FFFu));
+    for (int i = lane; 16 * i < nb; i += 32) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(src) + i);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int k = 0; k < 4; k++) {
+            const int rem = nb - 16 * i - 4 * k;   // bytes of this word that hold scales
+            const uint32_t x = rem >= 4 ? w[k] : (rem > 0 ? w[k] & ((1u << (8 * rem)) - 1u) : 0u);
+            if constexpr (KIND == RK_E4M3_MX32)
+                mx = max(mx, max(max(x & 0xFFu, (x >> 8) & 0xFFu), max((x >> 16) & 0xFFu, x >> 24)));
+            else
+                mx = max(mx, max(x & 0x7FFFu, (x >> 16) & 0x7FFFu));
         }
     }
-    mx = __reduce_max_sync(0xffffffffu, mx);
+    return mx;
+}
+
+// floor(log2) of a scale given as scale_bits_max bits (0 for 0).
+template <int KIND>
+__device__ __forceinline__ int scale_exp_of_bits(uint32_t mx) {
     if (mx == 0) return 0;
     if constexpr (KIND == RK_E4M3_MX32) return (int)mx - 127;
     else return (int)max(mx >> 10, 1u) - 15;   // fp16 exponent field (subnormals: 2^-14)
+}
+
+// The scale exponents of a (sequence, kv-head): floor(log2) of its largest K
+// and V scale over the cached tokens [0, Ls), the same in every thread of the
+// CTA.  Every tile of the sequence is dequantised as code x scale x 2^-e, so
+// every value lies below 2 x the largest code, and the 2^e goes back in fp32.
+// One pass over the scale rows (16 bytes per token for INT8 at head_dim 256),
+// once per CTA, while the ring's first copies are in flight.
+template <int KK, int KV, int D>
+__device__ void sequence_scale_exps(const PrefillParams& p, int b, int hh, int Ls, uint32_t* red, int* ek, int* ev) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr int NW = kPrefillThreads / 32;
+    uint32_t mk = 0, mv = 0;
+    const int np = (Ls + p.L.P - 1) / p.L.P;
+    // warp w takes 32 pages at a time (pages w*32 + 8*32*k + q), their ids loaded
+    // by the lanes at once; each page id then comes from a shuffle, so the
+    // scale loads of several pages are in flight together
+    for (int pg0 = warp * 32; pg0 < np; pg0 += NW * 32) {
+        int pid = -1;
+        if (pg0 + lane < np && pg0 + lane < p.max_pages) pid = p.block_table[(int64_t)b * p.max_pages + pg0 + lane];
+        if (pid < 0 || pid >= p.L.num_pages) pid = 0;   // recorded by the ring's copies
+        const int cnt = min(32, np - pg0);
+#pragma unroll 4
+        for (int q = 0; q < cnt; q++) {
+            const int id = __shfl_sync(0xffffffffu, pid, q);
+            const uint8_t* slab = p.slabs + ((int64_t)id * p.L.H + hh) * p.L.slab;
+            const int rows = min(p.L.P, Ls - (pg0 + q) * p.L.P);
+            if constexpr (scale_normalised(KK)) mk = max(mk, scale_bits_max<KK>(slab + p.L.off_ks, rows * p.L.ks, lane));
+            if constexpr (scale_normalised(KV)) mv = max(mv, scale_bits_max<KV>(slab + p.L.off_vs, rows * p.L.vs, lane));
+        }
+    }
+    mk = __reduce_max_sync(0xffffffffu, mk);
+    mv = __reduce_max_sync(0xffffffffu, mv);
+    __syncthreads();   // `red` may still be read by the previous block's epilogue
+    if (lane == 0) {
+        red[warp] = mk;
+        red[8 + warp] = mv;
+    }
+    __syncthreads();
+    for (int w = 0; w < kPrefillThreads / 32; w++) {
+        mk = max(mk, red[w]);
+        mv = max(mv, red[8 + w]);
+    }
+    *ek = scale_exp_of_bits<KK>(mk);
+    *ev = scale_exp_of_bits<KV>(mv);
 }
 
 // Stage the block's 128 query rows into sQ: row r is global row R0 + r of the
@@ -420,14 +474,29 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const Prefi
         if (!mbar_wait(bar, phase, abort_flag, p.wait_polls) && lane == 0) atomicOr(p.status, kStatusWaitTimeout);
     };
 
-    uint32_t seq = 0;   // key tiles consumed by this CTA: ring stage seq % stages, phase seq / stages
-    uint32_t rnd = 0;   // MMA rounds (one S and one O per tile): phase of barS and barO
-    for (int64_t jb = slot; jb < nblk; jb += p.slots) {
+    // key tiles of query block jb: those up to its largest position
+    auto block_tiles = [&](int64_t jb) {
         const int64_t R0 = (nblk - 1 - jb) * kPrefillRows;   // the heaviest block first
         const int64_t r_last = min(R0 + kPrefillRows, rows_total) - 1;
         const int pos_hi = Ls - n + (int)(r_last / p.G);        // largest position in the block
-        const int ntiles = pos_hi >= 0 ? pos_hi / T + 1 : 0;
-        if (tid == 0)
+        return pos_hi >= 0 ? pos_hi / T + 1 : 0;
+    };
+    // the first block's ring starts filling before the scale scan below
+    if (tid == 0)
+        for (int k = 0; k < p.stages && k < block_tiles(slot); k++) issue(k, k);
+
+    // the sequence's scale exponents (INT8, E4M3 row-256, MX)
+    int ek_seq = 0, ev_seq = 0;
+    if constexpr (scale_normalised(KK) || scale_normalised(KV))
+        sequence_scale_exps<KK, KV, D>(p, b, hh, Ls, reinterpret_cast<uint32_t*>(red), &ek_seq, &ev_seq);
+    const float kmul = pow2i(-ek_seq), vmul = pow2i(-ev_seq);
+
+    uint32_t seq = 0;   // key tiles consumed by this CTA: ring stage seq % stages, phase seq / stages
+    uint32_t rnd = 0;   // MMA rounds (one S and one O per tile): phase of barS and barO
+    for (int64_t jb = slot; jb < nblk; jb += p.slots) {
+        const int64_t R0 = (nblk - 1 - jb) * kPrefillRows;
+        const int ntiles = block_tiles(jb);
+        if (tid == 0 && jb != slot)
             for (int k = 0; k < p.stages && k < ntiles; k++) issue(seq + k, k);
         stage_q<D, KBF>(p, sQ, qrm, qrow0, hh, R0, rows_total, warp, lane);
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -439,13 +508,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const Prefi
         const int64_t gfirst = R0 + g4 * 32;
         const int gpos_min = gfirst + 31 < rows_total ? Ls - n + (int)(gfirst / p.G) : -1;
         float m_ref = -INFINITY, l_part = 0.f;
-        // value tiles enter scaled by 2^-eV (their own scale exponent); P carries
-        // 2^(eV - ev_ref) so that O stays in units of 2^ev_ref, a reference raised
-        // (O rescaled) when a tile's exponent exceeds it by more than 4
-        int ev_ref = 0;
-        bool ev_set = false;
         __syncthreads();   // q staged
-        const float qrow = qrm[r];
+        const float qm = p.q_mult * pow2i(ek_seq) * qrm[r];   // this row's score multiplier
 
         for (int k = 0; k < ntiles; k++, seq++, rnd++) {
             const int s = (int)(seq % (uint32_t)p.stages);
@@ -453,12 +517,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const Prefi
             wait_or_flag(smem_addr(&bars[s]), (seq / (uint32_t)p.stages) & 1u);
             const int t0 = k * T;
             const int valid = min(T, Ls - t0);
-            // the tile's scale exponents (every warp computes them from the stage)
-            int ek = 0, evt = 0;
-            if constexpr (scale_normalised(KK)) ek = tile_scale_exp<KK, D>(st + p.st_ks, valid, lane);
-            if constexpr (scale_normalised(KV)) evt = tile_scale_exp<KV, D>(st + p.st_vs, valid, lane);
             // keys first: S of this tile can start while the values are dequantised
-            dequant_tile<KK, D>(st, st + p.st_ks, sK, T, lgT, valid, tid, pow2i(-ek));
+            dequant_tile<KK, D>(st, st + p.st_ks, sK, T, lgT, valid, tid, kmul);
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncthreads();
             if (tid == 0 && !*abort_flag) {
@@ -474,24 +534,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const Prefi
                 wait_or_flag(barO, (rnd - 1) & 1u);
                 tc::fence_after();
             }
-            dequant_tile<KV, D>(st + p.st_vc, st + p.st_vs, sV, T, lgT, valid, tid, pow2i(-evt));
+            dequant_tile<KV, D>(st + p.st_vc, st + p.st_vs, sV, T, lgT, valid, tid, vmul);
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            // the value reference: set by the first tile, raised when this tile's
-            // exponent is more than 2^4 above it (the same decision in every thread)
-            float vcorr = 1.f;
-            bool vresc = false;
-            if constexpr (scale_normalised(KV)) {
-                if (!ev_set || evt > ev_ref + 4) {
-                    if (ev_set) {
-                        vcorr = pow2i(ev_ref - evt);
-                        vresc = true;
-                    }
-                    ev_ref = evt;
-                    ev_set = true;
-                }
-            }
-            const int dv = evt - ev_ref;   // <= 4: P of this tile carries 2^dv
-            const float qm = p.q_mult * pow2i(ek) * qrow;
 
             // ---- scores of this thread's row, columns [32 h, 32 h + 32) of the tile
             wait_or_flag(barS, rnd & 1u);
@@ -526,8 +570,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const Prefi
                 corr = ex2(m_ref - mt);
                 m_ref = mt;
             }
-            // P of this tile = 2^(s - m_ref + dv): the value tile's 2^dv is folded in
-            const float base = (m_ref == -INFINITY ? 0.f : m_ref) - (float)dv;
+            const float base = m_ref == -INFINITY ? 0.f : m_ref;
             float rs = 0.f;
             if (active) {
 #pragma unroll
@@ -543,10 +586,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const Prefi
                         *reinterpret_cast<uint4*>(sP + p_off(r, c0 + 8 * q8)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
                 }
             }
-            l_part = l_part * corr + rs * pow2i(-dv);
-            if (k > 0 && (vresc || __any_sync(0xffffffffu, resc))) {
+            l_part = l_part * corr + rs;
+            if (k > 0 && __any_sync(0xffffffffu, resc)) {
                 // O of this thread's row, columns [h D/2, h D/2 + D/2), times corr
-                corr *= vcorr;
 #pragma unroll 1
                 for (int cc = 0; cc < D / 2; cc += 32) {
                     uint32_t v[32];
@@ -582,7 +624,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const Prefi
         red[h * kPrefillRows + r] = l_part;
         __syncthreads();
         const float l = red[r] + red[kPrefillRows + r];
-        const float inv = l > 0.f ? p.o_mult / l * pow2i(ev_ref) : 0.f;   // O is in units of 2^ev_ref
+        const float inv = l > 0.f ? p.o_mult / l * pow2i(ev_seq) : 0.f;   // O is in units of 2^ev_seq
         float* so = sO + r * OST + h * (D / 2);
 #pragma unroll 1
         for (int cc = 0; cc < D / 2; cc += 32) {
