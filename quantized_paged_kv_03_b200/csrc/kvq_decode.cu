@@ -36,6 +36,8 @@
 //  * Rotated K: q is rotated by the same normalised Hadamard-256 (orthonormal,
 //    so q.k is unchanged).  Rotated V: the output is rotated back (the matrix
 //    is symmetric and its own inverse).
+#include <type_traits>
+
 #include "kvq_quant.cuh"
 
 namespace kvq {
@@ -83,9 +85,6 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
                  "l"(src), "r"(bytes), "r"(bar)
                  : "memory");
-}
-__device__ __forceinline__ void pair_sync(int id) {   // the two warps of a tile pair
-    asm volatile("bar.sync %0, 64;" ::"r"(id) : "memory");
 }
 
 __device__ __forceinline__ void mma_f16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
@@ -201,12 +200,10 @@ struct DecTraits {
     static constexpr int KNB = 4 * KCH * KBITS / 8;            // bytes per lane per K row load
     static constexpr int VNB = 4 * VCH * VBITS / 8;
     static constexpr int KCHUNKS = KSTEPS / KCH, VCHUNKS = DTILES / VCH;
-    static constexpr int KC_HALF = KCHUNKS / 2, VC_HALF = VCHUNKS / 2;   // per warp of a pair
     static constexpr int QS = (KK == RK_BF16RAW) ? 2 : 1;      // q split into hi (+ lo)
     static constexpr int KC = row_code_bytes(KK, D), KS = row_scale_bytes(KK, D);   // row bytes
     static constexpr int VC = row_code_bytes(KV, D), VS = row_scale_bytes(KV, D);
     static constexpr int EPL = D / 32;
-    static_assert(KCHUNKS % 2 == 0 && VCHUNKS % 2 == 0, "head_dim halves must hold whole chunks");
 };
 
 // Cursor over this CTA's page-heads: (sequence b, head pair hh = h*HB + hb, page).
@@ -422,41 +419,31 @@ __device__ __forceinline__ void merge_segment(const float* partials, void* out, 
     }
 }
 
-// Shared state of the stage producer (only the warp that issues a copy touches it).
-struct Producer {
-    Cursor c;
-    int issued;
-};
-
-// CTAs per SM a decode kernel is compiled for.  Three (24 warps, registers
-// capped at 80 per thread) where a 64-token page is small enough for three CTAs
-// to keep three stages each in shared memory and the head_dim-128 state fits
-// the cap; two otherwise (head_dim 256 needs the registers, BF16 pages are
-// 32 KB, and MXFP8's 128-token pages run faster whole at two CTAs than split
-// into 64-token units at three).
+// CTAs per SM a decode kernel is compiled for: two (16 warps, up to 128
+// registers per thread), which every format's full-head_dim accumulators need.
 __host__ __device__ constexpr int decode_ctas(int kk, int vk, int D) {
-    return (D == 128 && kk != RK_E4M3_MX32 &&
-            64 * (row_code_bytes(kk, D) + row_scale_bytes(kk, D) + row_code_bytes(vk, D) + row_scale_bytes(vk, D)) <=
-                20 * 1024)
-               ? 3
-               : 2;
+    (void)kk;
+    (void)vk;
+    (void)D;
+    return 2;
 }
 
-// The fused append (kvq_append_decode) of one sequence's newest token: warp 0
-// quantises its K row, warp 1 its V row, into the stage (row t of the unit)
-// and, when g is set, into the cache slab (row tp of the page).  Out of line:
-// it runs once per sequence, and keeping it out of the decode loop keeps the
-// loop's code compact.
+// The fused append (kvq_append_decode) of one sequence's newest token: role 0
+// quantises its K row, role 1 its V row, role 2 both, into the stage (row t of
+// the unit) and, when g is set, into the cache slab (row tp of the page).  Out
+// of line: it runs once per sequence, and keeping it out of the decode loop
+// keeps the loop's code compact.
 template <int KK, int KV, int D>
-__device__ __noinline__ void fused_append_rows(int warp, int lane, const uint16_t* k_src, const uint16_t* v_src,
+__device__ __noinline__ void fused_append_rows(int role, int lane, const uint16_t* k_src, const uint16_t* v_src,
                                                bool rot_k, bool rot_v, float k_scale, float v_scale, uint8_t* st,
                                                uint8_t* g, int t, int tp, int u_ks, int u_vc, int u_vs, int c_ks,
                                                int c_vc, int c_vs) {
     using T = DecTraits<KK, KV, D>;
-    if (warp == 0) {
+    if (role != 1) {
         quantize_row<KK, D>(k_src, rot_k, k_scale, st + t * T::KC, st + u_ks + t * T::KS, t, lane,
                             g ? g + tp * T::KC : nullptr, g ? g + c_ks + tp * T::KS : nullptr);
-    } else {
+    }
+    if (role != 0) {
         quantize_row<KV, D>(v_src, rot_v, v_scale, st + u_vc + t * T::VC, st + u_vs + t * T::VS, t, lane,
                             g ? g + c_vc + tp * T::VC : nullptr, g ? g + c_vs + tp * T::VS : nullptr);
     }
@@ -469,7 +456,6 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
     extern __shared__ __align__(128) uint8_t smem[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int r = lane >> 2, j = lane & 3;
-    const int tw = warp >> 1, hf = warp & 1;     // tile slot, head_dim half (the pair on two schedulers)
     const int H = p.L.H, P = p.L.P, HB = p.HB, HH = H * HB, B = p.B;
     const int64_t slab = p.L.slab;            // page slab stride in HBM
     const SpanLayout& U = p.U;                // what one stage holds
@@ -481,15 +467,16 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
     off += 8 * kMaxStages;
     int* rel = reinterpret_cast<int*>(smem + off);               // release count[stage]
     off += 4 * kMaxStages;
-    Producer* prod = reinterpret_cast<Producer*>(smem + off);
-    off += 32;
-    float* osm = reinterpret_cast<float*>(smem + off);   // [8][D]: q staging / output combine / score exchange
-    off += (8 * kOsmStride<D> * 4 > 8192 ? 8 * kOsmStride<D> * 4 : 8192);
-    float4* xbuf = reinterpret_cast<float4*>(osm);       // [2 parity][4 tiles][2 halves][32 lanes]
+    volatile int* tagv = reinterpret_cast<volatile int*>(smem + off);   // unit last issued into [stage]
+    off += 4 * kMaxStages;
+    int* iss = reinterpret_cast<int*>(smem + off);               // copies issued into [stage]
+    off += 4 * kMaxStages;
+    float* osm = reinterpret_cast<float*>(smem + off);   // [8][D]: output combine
+    off += 8 * kOsmStride<D> * 4;
     uint8_t* qst = smem + off;                           // q fragments of the segment (fp16 / bf16 hi, lo)
     off += 8 * (size_t)D * 2 * T::QS;
-    float* wml = reinterpret_cast<float*>(smem + off);   // [4 tile warps][m 8, l 8]
-    off += 4 * 16 * 4;
+    float* wml = reinterpret_cast<float*>(smem + off);   // [8 warps][m 8, l 8]
+    off += 8 * 16 * 4;
     float* fin = reinterpret_cast<float*>(smem + off);   // [m 8][l 8] of the merged segment
     off += 16 * 4;
     float* qhm = reinterpret_cast<float*>(smem + off);   // [8] score multiplier of each head of the block
@@ -576,17 +563,29 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
     auto pid_at = [&](const Cursor& c) {
         return checked(p.block_table[(int64_t)c.b * p.max_pages + (c.span >> U.lg_up)]);
     };
-    auto page_id = [&](int64_t w) {
+    // Where unit w (of the whole batch) comes from: (slab index << 2) | the
+    // unit's 64-token span within its page (for pages staged in spans).
+    const uint32_t span_mask = (1u << U.lg_up) - 1u;
+    auto unit_word = [&](const Cursor& c) {
+        return ((uint32_t)(pid_at(c) * H + c.h) << 2) | ((uint32_t)c.span & span_mask);
+    };
+    auto unit_src = [&](int k) {   // unit k of this CTA's range
+        if (k < p.pid_cap) return (uint32_t)pids[k];
         Cursor c;
-        cursor_locate(c, w, pref, B, HH, HB);
-        return pid_at(c);
+        cursor_locate(c, w0 + k, pref, B, HH, HB);
+        return unit_word(c);
     };
 
-    // ---- producer: the next unit into a free stage (one copy of a whole page
-    // slab, or the unit's rows of each of the slab's four arrays)
-    auto issue = [&](int s, int pid) {
-        Cursor& pc = prod->c;
-        const uint8_t* src = p.slabs + ((int64_t)pid * H + pc.h) * slab;
+    // ---- producer: unit k of the range into stage k % NS (one copy of a whole
+    // page slab, or the unit's rows of each of the slab's four arrays).  The
+    // warp groups release their units independently, so units are refilled
+    // out of order; tagv[s] records the unit a stage was last issued for, and a
+    // consumer waits on the stage's mbarrier only once the tag names its unit
+    // (the mbarrier's phase parity cannot tell a pending copy from a phase
+    // completed two uses ago).
+    auto issue = [&](int k, int s) {   // s == k % NS
+        const uint32_t us = unit_src(k);
+        const uint8_t* src = p.slabs + (int64_t)(us >> 2) * slab;
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         const uint32_t bar = smem_u32(&bars[s]);
         const uint32_t dst = smem_u32(smem + (size_t)s * U.bytes);
@@ -594,7 +593,7 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
             mbar_expect_tx(bar, (uint32_t)slab);
             bulk_g2s(dst, src, (uint32_t)slab, bar);
         } else {
-            const int64_t r0 = (int64_t)(pc.span & ((1 << U.lg_up) - 1)) * U.sp;
+            const int64_t r0 = (int64_t)(us & 3u) * U.sp;
             const uint32_t nk = U.sp * p.L.kc, nks = U.sp * p.L.ks, nv = U.sp * p.L.vc, nvs = U.sp * p.L.vs;
             mbar_expect_tx(bar, nk + nks + nv + nvs);
             bulk_g2s(dst, src + r0 * p.L.kc, nk, bar);
@@ -602,41 +601,49 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
             bulk_g2s(dst + (uint32_t)U.off_vc, src + p.L.off_vc + r0 * p.L.vc, nv, bar);
             if (nvs) bulk_g2s(dst + (uint32_t)U.off_vs, src + p.L.off_vs + r0 * p.L.vs, nvs, bar);
         }
-        cursor_next(pc, pref, B, HH, HB);
-        prod->issued++;
+        iss[s]++;
+        __threadfence_block();
+        tagv[s] = k;
     };
     // thread 0 starts the ring with its own block-table reads (all in flight at
-    // once) while the other threads preload the range's page ids
+    // once) while the other threads preload the range's unit sources
     if (tid == 0) {
         for (int s = 0; s < NS; s++) {
             mbar_init(smem_u32(&bars[s]), 1);
             rel[s] = 0;
+            iss[s] = 0;
+            tagv[s] = -1;
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        cursor_locate(prod->c, w0, pref, B, HH, HB);
-        prod->issued = 0;
-        Cursor c = prod->c;
+        Cursor c;
+        cursor_locate(c, w0, pref, B, HH, HB);
 #pragma unroll
         for (int s = 0; s < kMaxStages; s++) {
             if (s < NS && s < n) {
-                pids[s] = checked(p.block_table[(int64_t)c.b * p.max_pages + (c.span >> U.lg_up)]);
+                pids[s] = (int)unit_word(c);
                 cursor_next(c, pref, B, HH, HB);
             }
         }
-        for (int s = 0; s < NS && s < n; s++) issue(s, pids[s]);
+        for (int s = 0; s < NS && s < n; s++) issue(s, s);
     }
-    for (int k = NS + tid; k < n && k < p.pid_cap; k += kDecThreads) pids[k] = page_id(w0 + k);
+    for (int k = NS + tid; k < n && k < p.pid_cap; k += kDecThreads) {
+        Cursor c;
+        cursor_locate(c, w0 + k, pref, B, HH, HB);
+        pids[k] = (int)unit_word(c);
+    }
     __syncthreads();
 
-    // ---- consumer state (warp pair: tile slot tw, head_dim half hf)
-    Cursor cc;
-    cursor_locate(cc, w0, pref, B, HH, HB);
-    const int tiles = U.sp >> 4;    // 16-token tiles per unit
-    int s = 0;                   // stage of page i
-    uint32_t ph = 0;             // mbarrier phase of that stage's current use
+    // ---- consumer layout.  A warp owns a 16-token tile over all of head_dim.
+    // A unit's tiles go to a group of wpu warps; the CTA's ngrp groups take a
+    // segment's units in turn (unit i + g, i + g + ngrp, ... to group g), so
+    // several units are in flight and every warp's state covers the whole
+    // segment.
+    const int tiles = U.sp >> 4;                  // 16-token tiles per unit
+    const int wpu = tiles < 8 ? tiles : 8;        // warps per unit
+    const int ngrp = (kDecThreads / 32) / wpu;    // units in flight
+    const int grp = warp / wpu, tile = warp - grp * wpu;
     int seq_len = 0;
-    uint32_t qf[T::KSTEPS / 2][T::QS][2];
-    float o[T::DTILES / 2][4];
+    float o[T::DTILES][4];
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
     float hm0 = 1.f, hm1 = 1.f;   // score multipliers of heads 2j, 2j + 1 (q's power of two, K tensor scale)
     // V scales folded into P' (FP8 row-256, INT8, MX V): P' = P * (scale * 2^-ve),
@@ -645,380 +652,372 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
     // keeps P' inside fp16's normal range whatever the magnitude of V.
     int ve = 0;
     float vmul = 1.f, vthr = 0.f;   // 2^-ve; 2^(ve + 4), 0 before the segment's first nonzero scale
-    bool seg_first = true;     // segment began at this CTA's first page
-    int xpar = 0;              // score-exchange buffer parity
 
-    // Per-lane byte offsets inside a stage, fixed for the whole kernel: lane
-    // (r, j) reads token rows r and r + 8 of a tile (same chunk permutation, since
-    // the permutation depends on the row modulo 4) at the chunks of its half.
+    // Per-lane byte offsets inside a stage: lane (r, j) reads token rows r and
+    // r + 8 of a tile (same chunk permutation, since the permutation depends on
+    // the row modulo 4), chunk cl at 4 * KCH * j within it.
     const int swk = row_swizzle(KK, D, r), swv = row_swizzle(KV, D, r);
-    uint32_t koff[T::KC_HALF], voff[T::VC_HALF], ksoff[T::KC_HALF], vsoff[T::VC_HALF];
-#pragma unroll
-    for (int cl = 0; cl < T::KC_HALF; cl++) {
-        const int c = hf * T::KC_HALF + cl;
-        koff[cl] = r * T::KC + phys_byte((T::KCW * c + 4 * T::KCH * j) * T::KBITS / 8, swk);
-        if constexpr (KK == RK_E2M1_G16) ksoff[cl] = r * T::KS + (T::KCW * c + 16 * j) / 16;
-        else if constexpr (KK == RK_INT8_G64) ksoff[cl] = r * T::KS + 2 * c;
-        else if constexpr (KK == RK_E4M3_MX32) ksoff[cl] = r * T::KS + c;
-        else ksoff[cl] = r * T::KS;
-    }
-#pragma unroll
-    for (int cl = 0; cl < T::VC_HALF; cl++) {
-        const int c = hf * T::VC_HALF + cl;
-        voff[cl] = r * T::VC + phys_byte((T::VCW * c + 4 * T::VCH * j) * T::VBITS / 8, swv);
-        if constexpr (KV == RK_E2M1_G16) vsoff[cl] = r * T::VS + (T::VCW * c + 16 * j) / 16;
-        else if constexpr (KV == RK_INT8_G64) vsoff[cl] = r * T::VS + 2 * c;
-        else if constexpr (KV == RK_E4M3_MX32) vsoff[cl] = r * T::VS + c;
-        else vsoff[cl] = r * T::VS;
-    }
+    auto koff = [&](int cl) { return (uint32_t)(r * T::KC + phys_byte((T::KCW * cl + 4 * T::KCH * j) * T::KBITS / 8, swk)); };
+    auto voff = [&](int cl) { return (uint32_t)(r * T::VC + phys_byte((T::VCW * cl + 4 * T::VCH * j) * T::VBITS / 8, swv)); };
+    auto ksoff = [&](int cl) {
+        if constexpr (KK == RK_E2M1_G16) return (uint32_t)(r * T::KS + (T::KCW * cl + 16 * j) / 16);
+        else if constexpr (KK == RK_INT8_G64) return (uint32_t)(r * T::KS + 2 * cl);
+        else if constexpr (KK == RK_E4M3_MX32) return (uint32_t)(r * T::KS + cl);
+        else return (uint32_t)(r * T::KS);
+    };
+    auto vsoff = [&](int cl) {
+        if constexpr (KV == RK_E2M1_G16) return (uint32_t)(r * T::VS + (T::VCW * cl + 16 * j) / 16);
+        else if constexpr (KV == RK_INT8_G64) return (uint32_t)(r * T::VS + 2 * cl);
+        else if constexpr (KV == RK_E4M3_MX32) return (uint32_t)(r * T::VS + cl);
+        else return (uint32_t)(r * T::VS);
+    };
     const uint32_t off_ks = (uint32_t)U.off_ks, off_vc = (uint32_t)U.off_vc, off_vs = (uint32_t)U.off_vs;
-    float4* xmine = xbuf + (tw * 2 + hf) * 32 + lane;          // parity 0; parity 1 is +8*32
-    const float4* xother = xbuf + (tw * 2 + (hf ^ 1)) * 32 + lane;
 
-    for (int i = 0; i < n; i++) {
+    Cursor cc;
+    cursor_locate(cc, w0, pref, B, HH, HB);
+    for (int i = 0; i < n;) {
         const int b = cc.b, h = cc.h, hb = cc.hb;
-        if (i == 0 || cc.span == 0) {
-            // ---- segment start: q rows of this 8-head block, rotated and scaled
-            seg_first = (i == 0);
-            seq_len = p.seq_lens[b];
-            {
-                // warp w stages head w of the block, already in the MMA fragment
-                // order: for k-step st, lane group j, head n, the 4 values of that
-                // lane's slice as fp16 pairs (hi, and lo for a bf16 split)
-                const int gq = hb * 8 + warp;
-                float x[8];
-                if (gq < p.G) {
-                    const uint16_t* qrow = p.q + ((int64_t)b * p.Hq + h * p.G + gq) * D + lane * T::EPL;
-                    uint32_t raw[4];
-                    if constexpr (T::EPL == 8) {
-                        const uint4 v = *reinterpret_cast<const uint4*>(qrow);
-                        raw[0] = v.x; raw[1] = v.y; raw[2] = v.z; raw[3] = v.w;
-                    } else {
-                        const uint2 v = *reinterpret_cast<const uint2*>(qrow);
-                        raw[0] = v.x; raw[1] = v.y; raw[2] = raw[3] = 0;
+        const int span0 = cc.span, nspans = cc.nspans;
+        const int seg_n = min(nspans - span0, n - i);   // this segment's units in the range
+        const bool seg_first = (i == 0);
+        seq_len = p.seq_lens[b];
+        {
+            // ---- segment start: q rows of this 8-head block, rotated and scaled.
+            // Warp w stages head w, already in the MMA fragment order: for
+            // k-step st, lane group j, head n, the 4 values of that lane's slice
+            // as fp16 pairs (hi, and lo for a bf16 split).
+            const int gq = hb * 8 + warp;
+            float x[8];
+            if (gq < p.G) {
+                const uint16_t* qrow = p.q + ((int64_t)b * p.Hq + h * p.G + gq) * D + lane * T::EPL;
+                uint32_t raw[4];
+                if constexpr (T::EPL == 8) {
+                    const uint4 v = *reinterpret_cast<const uint4*>(qrow);
+                    raw[0] = v.x; raw[1] = v.y; raw[2] = v.z; raw[3] = v.w;
+                } else {
+                    const uint2 v = *reinterpret_cast<const uint2*>(qrow);
+                    raw[0] = v.x; raw[1] = v.y; raw[2] = raw[3] = 0;
+                }
+#pragma unroll
+                for (int e = 0; e < T::EPL; e++) x[e] = bf16_bits_to_f32((raw[e >> 1] >> ((e & 1) * 16)) & 0xFFFFu);
+                if constexpr (D == 256) {
+                    if (p.rot_k) {
+                        Row8 y;
+#pragma unroll
+                        for (int e = 0; e < 8; e++) y.v[e] = x[e];
+                        y = fwht256_row(y, lane);
+#pragma unroll
+                        for (int e = 0; e < 8; e++) x[e] = y.v[e];
                     }
+                }
+                // q x softmax scale x log2(e), normalised by a power of two so
+                // that its largest element lies in [1, 2): fp16 keeps full
+                // precision whatever q's magnitude; the 2^e returns in the
+                // fp32 scores (with the K tensor scale, for FP8 per tensor)
+                float amax = 0.f;
 #pragma unroll
-                    for (int e = 0; e < T::EPL; e++) x[e] = bf16_bits_to_f32((raw[e >> 1] >> ((e & 1) * 16)) & 0xFFFFu);
-                    if constexpr (D == 256) {
-                        if (p.rot_k) {
-                            Row8 y;
+                for (int e = 0; e < T::EPL; e++) {
+                    x[e] *= p.q_mult;
+                    amax = fmaxf(amax, fabsf(x[e]));
+                }
+                amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(amax)));
+                const int eq = amax > 0.f ? exp2_floor(amax) : 0;
+                const float nq = pow2i(-eq);
 #pragma unroll
-                            for (int e = 0; e < 8; e++) y.v[e] = x[e];
-                            y = fwht256_row(y, lane);
+                for (int e = 0; e < T::EPL; e++) x[e] *= nq;
+                if (lane == 0) qhm[warp] = pow2i(eq) * p.k_tmult;
+            } else {
 #pragma unroll
-                            for (int e = 0; e < 8; e++) x[e] = y.v[e];
+                for (int e = 0; e < T::EPL; e++) x[e] = 0.f;
+                if (lane == 0) qhm[warp] = 0.f;
+            }
+#pragma unroll
+            for (int g4 = 0; g4 < T::EPL / 4; g4++) {
+                const int d0 = lane * T::EPL + 4 * g4;
+                const int c = d0 / T::KCW, rem = d0 % T::KCW;
+                const int jj = rem / (4 * T::KCH), ks = (rem % (4 * T::KCH)) / 4;
+                const int st = c * T::KCH + ks;
+                const float* v = x + 4 * g4;
+                const int slot = (st * 4 + jj) * 8 + warp;
+                if constexpr (T::QS == 2) {
+                    float lo[4];
+#pragma unroll
+                    for (int e = 0; e < 4; e++) lo[e] = v[e] - __bfloat162float(__float2bfloat16_rn(v[e]));
+                    reinterpret_cast<uint4*>(qst)[slot] = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]),
+                                                                     pack_bf16(lo[0], lo[1]), pack_bf16(lo[2], lo[3]));
+                } else {
+                    reinterpret_cast<uint2*>(qst)[slot] = make_uint2(pack_f16(v[0], v[1]), pack_f16(v[2], v[3]));
+                }
+            }
+        }
+        __syncthreads();
+        hm0 = qhm[2 * j];
+        hm1 = qhm[2 * j + 1];
+#pragma unroll
+        for (int u = 0; u < T::DTILES; u++) o[u][0] = o[u][1] = o[u][2] = o[u][3] = 0.f;
+        m0 = m1 = -INFINITY;
+        l0 = l1 = 0.f;
+        ve = 0;
+        vmul = 1.f;
+        vthr = 0.f;
+
+        // ---- this group's units of the segment
+        // the group's first unit of the segment: its stage and mbarrier phase
+        // (one division per segment; per unit they advance by ngrp)
+        int s = (i + grp) % NS;
+        uint32_t ph = (uint32_t)((i + grp) / NS) & 1u;
+        for (int u = i + grp; u < i + seg_n; u += ngrp) {
+            const int span = span0 + (u - i);
+            {
+                // wait until the stage was issued for this unit, then for its data
+                long it = 0;
+                while (tagv[s] != u && !*abort_flag) {
+                    if (++it > p.wait_polls) {
+                        *abort_flag = 1;
+                        break;
+                    }
+                }
+                (void)mbar_wait(smem_u32(&bars[s]), ph, abort_flag, p.wait_polls);
+            }
+            const uint32_t stg = (uint32_t)s * (uint32_t)U.bytes;   // byte offset of the stage
+
+            if (FUSED && span == nspans - 1) {
+                // fused append: the sequence's newest token (position seq_len - 1) lies
+                // in its last unit.  Quantise it into this stage (row t of the unit),
+                // over whatever the copy brought, and into the cache (row tp of the
+                // page; one head block writes the cache).  t and tp differ by a
+                // multiple of 64, so the row's chunk permutation is the same.
+                const int t = (seq_len - 1) - span * U.sp;
+                const int tp = t + (span & ((1 << U.lg_up) - 1)) * U.sp;
+                const int role = wpu >= 2 ? tile : 2;   // 0: K row, 1: V row, 2: both
+                if (role <= 2) {
+                    uint8_t* g = (hb == 0) ? p.slabs + (int64_t)(unit_src(u) >> 2) * slab : nullptr;
+                    const int64_t row = (int64_t)b * H + h;
+                    fused_append_rows<KK, KV, D>(role, lane, p.k_new + row * D, p.v_new + row * D, p.rot_k, p.rot_v,
+                                                 p.k_scale, p.v_scale, smem + stg, g, t, tp, (int)off_ks, (int)off_vc,
+                                                 (int)off_vs, (int)p.L.off_ks, (int)p.L.off_vc, (int)p.L.off_vs);
+                }
+                if (wpu > 1) asm volatile("bar.sync %0, %1;" ::"r"(1 + grp), "r"(wpu * 32) : "memory");
+                else __syncwarp();
+            }
+
+            for (int mt = tile; mt < tiles; mt += wpu) {
+                const int valid = seq_len - (span * U.sp + mt * 16);
+                if (valid <= 0) break;
+                const uint32_t kt = stg + mt * 16 * T::KC, kst = stg + off_ks + mt * 16 * T::KS;
+                const uint32_t vt = stg + off_vc + mt * 16 * T::VC, vst = stg + off_vs + mt * 16 * T::VS;
+                // ---------- S^T = K q^T over all of head_dim (tokens as M, heads as N)
+                float sc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int cl = 0; cl < T::KCHUNKS; cl++) {
+                    uint32_t xa[2 * T::KCH], xb[2 * T::KCH];
+                    slice_f16<KK, T::KNB, T::KCH>(lds_bytes<T::KNB>(smem + kt, koff(cl)), xa);
+                    slice_f16<KK, T::KNB, T::KCH>(lds_bytes<T::KNB>(smem + kt, koff(cl) + 8 * T::KC), xb);
+                    if constexpr (KK == RK_E2M1_G16) {
+                        const uint32_t sa = f16_splat(dec_e4m3x2_f16x2(smem[kst + ksoff(cl)]));
+                        const uint32_t sb = f16_splat(dec_e4m3x2_f16x2(smem[kst + ksoff(cl) + 8 * T::KS]));
+#pragma unroll
+                        for (int e = 0; e < 2 * T::KCH; e++) {
+                            xa[e] = hmul2(xa[e], sa);
+                            xb[e] = hmul2(xb[e], sb);
                         }
                     }
-                    // q x softmax scale x log2(e), normalised by a power of two so
-                    // that its largest element lies in [1, 2): fp16 keeps full
-                    // precision whatever q's magnitude; the 2^e returns in the
-                    // fp32 scores (with the K tensor scale, for FP8 per tensor)
-                    float amax = 0.f;
+                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                    for (int e = 0; e < T::EPL; e++) {
-                        x[e] *= p.q_mult;
-                        amax = fmaxf(amax, fabsf(x[e]));
+                    for (int ks = 0; ks < T::KCH; ks++) {
+                        const int sl = cl * T::KCH + ks;
+                        const uint32_t a[4] = {xa[2 * ks], xb[2 * ks], xa[2 * ks + 1], xb[2 * ks + 1]};
+                        if constexpr (T::QS == 2) {
+                            const uint4 qv = reinterpret_cast<const uint4*>(qst)[(sl * 4 + j) * 8 + r];
+                            mma_bf16(acc, a, qv.x, qv.y);
+                            mma_bf16(acc, a, qv.z, qv.w);
+                        } else {
+                            const uint2 qv = reinterpret_cast<const uint2*>(qst)[(sl * 4 + j) * 8 + r];
+                            mma_f16(acc, a, qv.x, qv.y);
+                        }
                     }
-                    amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(amax)));
-                    const int eq = amax > 0.f ? exp2_floor(amax) : 0;
-                    const float nq = pow2i(-eq);
-#pragma unroll
-                    for (int e = 0; e < T::EPL; e++) x[e] *= nq;
-                    if (lane == 0) qhm[warp] = pow2i(eq) * p.k_tmult;
-                } else {
-#pragma unroll
-                    for (int e = 0; e < T::EPL; e++) x[e] = 0.f;
-                    if (lane == 0) qhm[warp] = 0.f;
-                }
-#pragma unroll
-                for (int g4 = 0; g4 < T::EPL / 4; g4++) {
-                    const int d0 = lane * T::EPL + 4 * g4;
-                    const int c = d0 / T::KCW, rem = d0 % T::KCW;
-                    const int jj = rem / (4 * T::KCH), ks = (rem % (4 * T::KCH)) / 4;
-                    const int st = c * T::KCH + ks;
-                    const float* v = x + 4 * g4;
-                    const int slot = (st * 4 + jj) * 8 + warp;
-                    if constexpr (T::QS == 2) {
-                        float lo[4];
-#pragma unroll
-                        for (int e = 0; e < 4; e++) lo[e] = v[e] - __bfloat162float(__float2bfloat16_rn(v[e]));
-                        reinterpret_cast<uint4*>(qst)[slot] = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]),
-                                                                         pack_bf16(lo[0], lo[1]), pack_bf16(lo[2], lo[3]));
+                    if constexpr (KK == RK_INT8_G64 || KK == RK_E4M3_MX32) {
+                        float fa, fb;
+                        if constexpr (KK == RK_INT8_G64) {
+                            fa = f16_bits_to_f32(*reinterpret_cast<const uint16_t*>(smem + kst + ksoff(cl)));
+                            fb = f16_bits_to_f32(*reinterpret_cast<const uint16_t*>(smem + kst + ksoff(cl) + 8 * T::KS));
+                        } else {
+                            fa = ue8m0_to_f32(smem[kst + ksoff(cl)]);
+                            fb = ue8m0_to_f32(smem[kst + ksoff(cl) + 8 * T::KS]);
+                        }
+                        sc[0] = fmaf(acc[0], fa, sc[0]);
+                        sc[1] = fmaf(acc[1], fa, sc[1]);
+                        sc[2] = fmaf(acc[2], fb, sc[2]);
+                        sc[3] = fmaf(acc[3], fb, sc[3]);
                     } else {
-                        reinterpret_cast<uint2*>(qst)[slot] = make_uint2(pack_f16(v[0], v[1]), pack_f16(v[2], v[3]));
+                        sc[0] += acc[0]; sc[1] += acc[1]; sc[2] += acc[2]; sc[3] += acc[3];
                     }
                 }
-            }
-            __syncthreads();
-#pragma unroll
-            for (int sl = 0; sl < T::KSTEPS / 2; sl++) {
-                const int slot = ((hf * (T::KSTEPS / 2) + sl) * 4 + j) * 8 + r;
-                if constexpr (T::QS == 2) {
-                    const uint4 v = reinterpret_cast<const uint4*>(qst)[slot];
-                    qf[sl][0][0] = v.x; qf[sl][0][1] = v.y;
-                    qf[sl][T::QS - 1][0] = v.z; qf[sl][T::QS - 1][1] = v.w;
-                } else {
-                    const uint2 v = reinterpret_cast<const uint2*>(qst)[slot];
-                    qf[sl][0][0] = v.x; qf[sl][0][1] = v.y;
+                if constexpr (KK == RK_E4M3_ROW256) {
+                    const float fa = f16_bits_to_f32(*reinterpret_cast<const uint16_t*>(smem + kst + ksoff(0)));
+                    const float fb = f16_bits_to_f32(*reinterpret_cast<const uint16_t*>(smem + kst + ksoff(0) + 8 * T::KS));
+                    sc[0] *= fa; sc[1] *= fa; sc[2] *= fb; sc[3] *= fb;
                 }
-            }
-            hm0 = qhm[2 * j];
-            hm1 = qhm[2 * j + 1];
-#pragma unroll
-            for (int u = 0; u < T::DTILES / 2; u++) o[u][0] = o[u][1] = o[u][2] = o[u][3] = 0.f;
-            m0 = m1 = -INFINITY;
-            l0 = l1 = 0.f;
-            ve = 0;
-            vmul = 1.f;
-            vthr = 0.f;
-        }
+                // q's power of two (and the K tensor scale) back into the fp32 scores
+                sc[0] *= hm0; sc[1] *= hm1; sc[2] *= hm0; sc[3] *= hm1;
+                const bool oka = r < valid, okb = r + 8 < valid;
+                if (!oka) sc[0] = sc[1] = -INFINITY;
+                if (!okb) sc[2] = sc[3] = -INFINITY;
 
-        // wait for the slab
-        (void)mbar_wait(smem_u32(&bars[s]), ph, abort_flag, p.wait_polls);
+                // ---------- online softmax (log2 domain), heads 2j and 2j+1.  The
+                // running max is raised (with a warp-wide reduction and a rescale of
+                // the accumulators) only when a score exceeds it by more than 2^3;
+                // otherwise weights up to 8 are kept as they are.
+                {
+                    const float x0 = fmaxf(sc[0], sc[2]), x1 = fmaxf(sc[1], sc[3]);
+                    if (__any_sync(0xffffffffu, (x0 > m0 + 3.f) || (x1 > m1 + 3.f))) {
+                        float y0 = x0, y1 = x1;
+#pragma unroll
+                        for (int m = 4; m < 32; m <<= 1) {
+                            y0 = fmaxf(y0, __shfl_xor_sync(0xffffffffu, y0, m));
+                            y1 = fmaxf(y1, __shfl_xor_sync(0xffffffffu, y1, m));
+                        }
+                        const float n0 = fmaxf(m0, y0), n1 = fmaxf(m1, y1);
+                        const float a0 = (m0 == -INFINITY) ? 0.f : fast_exp2(m0 - n0);
+                        const float a1 = (m1 == -INFINITY) ? 0.f : fast_exp2(m1 - n1);
+#pragma unroll
+                        for (int u2 = 0; u2 < T::DTILES; u2++) {
+                            o[u2][0] *= a0; o[u2][1] *= a1; o[u2][2] *= a0; o[u2][3] *= a1;
+                        }
+                        l0 *= a0;
+                        l1 *= a1;
+                        m0 = n0;
+                        m1 = n1;
+                    }
+                }
+                const float r0 = (m0 == -INFINITY) ? 0.f : m0, r1 = (m1 == -INFINITY) ? 0.f : m1;
+                const float p0 = fast_exp2(sc[0] - r0), p1 = fast_exp2(sc[1] - r1);
+                const float p2 = fast_exp2(sc[2] - r0), p3 = fast_exp2(sc[3] - r1);
+                l0 += p0 + p2;
+                l1 += p1 + p3;
 
-        // ---- this pair's 16-token tiles of the page
-        const uint32_t stg = (uint32_t)s * (uint32_t)U.bytes;   // byte offset of the stage
+                // ---------- O^T += V^T P^T over all of head_dim
+                // rows past seq_len hold bytes never written: keep them out of the
+                // product entirely (their P is 0, but 0 x NaN would still be NaN)
+                const bool partial = valid < 16;
+                uint32_t pb0 = 0, pb1 = 0;   // P'^T fragment (B operand)
+                // V scales folded into P': this lane's rows r and r + 8, one per
+                // chunk (INT8, MX) or one per row (FP8 row-256), rows past seq_len 0
+                constexpr int NVS = VFOLD ? (KV == RK_E4M3_ROW256 ? 1 : T::VCHUNKS) : 1;
+                float vfa[NVS], vfb[NVS];
+                if constexpr (VFOLD) {
+                    float smax = 0.f;
+#pragma unroll
+                    for (int c = 0; c < NVS; c++) {
+                        if constexpr (KV == RK_E4M3_MX32) {
+                            vfa[c] = ue8m0_to_f32(smem[vst + vsoff(c)]);
+                            vfb[c] = ue8m0_to_f32(smem[vst + vsoff(c) + 8 * T::VS]);
+                        } else {
+                            vfa[c] = f16_bits_to_f32(*reinterpret_cast<const uint16_t*>(smem + vst + vsoff(c)));
+                            vfb[c] = f16_bits_to_f32(*reinterpret_cast<const uint16_t*>(smem + vst + vsoff(c) + 8 * T::VS));
+                        }
+                        vfa[c] = oka ? vfa[c] : 0.f;
+                        vfb[c] = okb ? vfb[c] : 0.f;
+                        smax = fmaxf(smax, fmaxf(vfa[c], vfb[c]));
+                    }
+                    if (__any_sync(0xffffffffu, smax > vthr)) {
+                        // raise the reference to the warp's largest scale (an exact power of two)
+                        const int en =
+                            exp2_floor(__uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(smax))));
+                        const float f = vthr > 0.f ? pow2i(ve - en) : 1.f;
+#pragma unroll
+                        for (int u2 = 0; u2 < T::DTILES; u2++) {
+                            o[u2][0] *= f; o[u2][1] *= f; o[u2][2] *= f; o[u2][3] *= f;
+                        }
+                        ve = en;
+                        vmul = pow2i(-en);
+                        vthr = pow2i(en + 4);
+                    }
+#pragma unroll
+                    for (int c = 0; c < NVS; c++) {
+                        vfa[c] *= vmul;
+                        vfb[c] *= vmul;
+                    }
+                }
+                if constexpr (KV == RK_E4M3_ROW256) {
+                    pb0 = movtrans(pack_f16(p0 * vfa[0], p1 * vfa[0]));
+                    pb1 = movtrans(pack_f16(p2 * vfb[0], p3 * vfb[0]));
+                } else if constexpr (!VFOLD) {
+                    pb0 = movtrans(pack_f16(p0, p1));
+                    pb1 = movtrans(pack_f16(p2, p3));
+                }
+#pragma unroll
+                for (int cl = 0; cl < T::VCHUNKS; cl++) {
+                    if constexpr (KV == RK_INT8_G64 || KV == RK_E4M3_MX32) {
+                        pb0 = movtrans(pack_f16(p0 * vfa[cl], p1 * vfa[cl]));
+                        pb1 = movtrans(pack_f16(p2 * vfb[cl], p3 * vfb[cl]));
+                    }
+                    uint32_t xa[2 * T::VCH], xb[2 * T::VCH];
+                    slice_f16<KV, T::VNB, T::VCH>(lds_bytes<T::VNB>(smem + vt, voff(cl)), xa);
+                    slice_f16<KV, T::VNB, T::VCH>(lds_bytes<T::VNB>(smem + vt, voff(cl) + 8 * T::VC), xb);
+                    if constexpr (KV == RK_E2M1_G16) {
+                        const uint32_t sa = f16_splat(dec_e4m3x2_f16x2(smem[vst + vsoff(cl)]));
+                        const uint32_t sb = f16_splat(dec_e4m3x2_f16x2(smem[vst + vsoff(cl) + 8 * T::VS]));
+#pragma unroll
+                        for (int e = 0; e < 2 * T::VCH; e++) {
+                            xa[e] = hmul2(xa[e], sa);
+                            xb[e] = hmul2(xb[e], sb);
+                        }
+                    }
+                    if (partial) {
+#pragma unroll
+                        for (int e = 0; e < 2 * T::VCH; e++) {
+                            xa[e] = oka ? xa[e] : 0u;
+                            xb[e] = okb ? xb[e] : 0u;
+                        }
+                    }
+#pragma unroll
+                    for (int u2 = 0; u2 < T::VCH; u2++) {
+                        const uint32_t a[4] = {movtrans(xa[2 * u2]), movtrans(xa[2 * u2 + 1]), movtrans(xb[2 * u2]),
+                                               movtrans(xb[2 * u2 + 1])};
+                        mma_f16(o[cl * T::VCH + u2], a, pb0, pb1);
+                    }
+                }
+            }
 
-        if (FUSED && cc.span == cc.nspans - 1) {
-            // fused append: the sequence's newest token (position seq_len - 1) lies
-            // in its last unit.  Quantise it into this stage (row t of the unit),
-            // over whatever the copy brought, and into the cache (row tp of the
-            // page; one head block writes the cache).  t and tp differ by a
-            // multiple of 64, so the row's chunk permutation is the same.
-            const int t = (seq_len - 1) - cc.span * U.sp;
-            const int tp = t + (cc.span & ((1 << U.lg_up) - 1)) * U.sp;
-            if (warp < 2) {
-                const int pid = (i < p.pid_cap) ? pids[i] : page_id(w0 + i);
-                uint8_t* g = (hb == 0) ? p.slabs + ((int64_t)pid * H + h) * slab : nullptr;
-                const int64_t row = (int64_t)b * H + h;
-                fused_append_rows<KK, KV, D>(warp, lane, p.k_new + row * D, p.v_new + row * D, p.rot_k, p.rot_v,
-                                             p.k_scale, p.v_scale, smem + stg, g, t, tp, (int)off_ks, (int)off_vc,
-                                             (int)off_vs, (int)p.L.off_ks, (int)p.L.off_vc, (int)p.L.off_vs);
-            }
-            asm volatile("bar.sync 5, %0;" ::"r"(kDecThreads) : "memory");
-        }
-        for (int mt = tw; mt < tiles; mt += 4) {
-            const int valid = seq_len - (cc.span * U.sp + mt * 16);
-            if (valid <= 0) break;   // same decision in both warps of the pair
-            const uint32_t kt = stg + mt * 16 * T::KC, kst = stg + off_ks + mt * 16 * T::KS;
-            const uint32_t vt = stg + off_vc + mt * 16 * T::VC, vst = stg + off_vs + mt * 16 * T::VS;
-            // ---------- partial S^T = K q^T over this warp's half of head_dim
-            float sc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int cl = 0; cl < T::KC_HALF; cl++) {
-                uint32_t xa[2 * T::KCH], xb[2 * T::KCH];
-                slice_f16<KK, T::KNB, T::KCH>(lds_bytes<T::KNB>(smem + kt, koff[cl]), xa);
-                slice_f16<KK, T::KNB, T::KCH>(lds_bytes<T::KNB>(smem + kt, koff[cl] + 8 * T::KC), xb);
-                if constexpr (KK == RK_E2M1_G16) {
-                    const uint32_t sa = f16_splat(dec_e4m3x2_f16x2(smem[kst + ksoff[cl]]));
-                    const uint32_t sb = f16_splat(dec_e4m3x2_f16x2(smem[kst + ksoff[cl] + 8 * T::KS]));
-#pragma unroll
-                    for (int e = 0; e < 2 * T::KCH; e++) {
-                        xa[e] = hmul2(xa[e], sa);
-                        xb[e] = hmul2(xb[e], sb);
-                    }
-                }
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int ks = 0; ks < T::KCH; ks++) {
-                    const int sl = cl * T::KCH + ks;
-                    const uint32_t a[4] = {xa[2 * ks], xb[2 * ks], xa[2 * ks + 1], xb[2 * ks + 1]};
-#pragma unroll
-                    for (int qs = 0; qs < T::QS; qs++) {
-                        if constexpr (KK == RK_BF16RAW) mma_bf16(acc, a, qf[sl][qs][0], qf[sl][qs][1]);
-                        else mma_f16(acc, a, qf[sl][qs][0], qf[sl][qs][1]);
-                    }
-                }
-                if constexpr (KK == RK_INT8_G64 || KK == RK_E4M3_MX32) {
-                    float fa, fb;
-                    if constexpr (KK == RK_INT8_G64) {
-                        fa = f16_bits_to_f32(*reinterpret_cast<const uint16_t*>(smem + kst + ksoff[cl]));
-                        fb = f16_bits_to_f32(*reinterpret_cast<const uint16_t*>(smem + kst + ksoff[cl] + 8 * T::KS));
-                    } else {
-                        fa = ue8m0_to_f32(smem[kst + ksoff[cl]]);
-                        fb = ue8m0_to_f32(smem[kst + ksoff[cl] + 8 * T::KS]);
-                    }
-                    sc[0] = fmaf(acc[0], fa, sc[0]);
-                    sc[1] = fmaf(acc[1], fa, sc[1]);
-                    sc[2] = fmaf(acc[2], fb, sc[2]);
-                    sc[3] = fmaf(acc[3], fb, sc[3]);
-                } else {
-                    sc[0] += acc[0]; sc[1] += acc[1]; sc[2] += acc[2]; sc[3] += acc[3];
+            // ---- release stage s; the last warp of the group to release it refills
+            // it.  The warp's reads of the stage have all returned (their values
+            // fed the MMAs above), so the count needs no fence before it.
+            __syncwarp();
+            if (lane == 0) {
+                const int old = atomicAdd(&rel[s], 1);
+                if (old == wpu - 1) {
+                    rel[s] = 0;
+                    __threadfence_block();
+                    if (u + NS < n && !*abort_flag) issue(u + NS, s);
                 }
             }
-            // ---------- add the two halves (same order in both warps: identical sums)
-            {
-                *(xmine + xpar * 256) = make_float4(sc[0], sc[1], sc[2], sc[3]);
-                pair_sync(1 + tw);
-                const float4 ot = *(xother + xpar * 256);
-                if (hf == 0) {
-                    sc[0] += ot.x; sc[1] += ot.y; sc[2] += ot.z; sc[3] += ot.w;
-                } else {
-                    sc[0] = ot.x + sc[0]; sc[1] = ot.y + sc[1]; sc[2] = ot.z + sc[2]; sc[3] = ot.w + sc[3];
-                }
-                xpar ^= 1;
-            }
-            if constexpr (KK == RK_E4M3_ROW256) {
-                const float fa = f16_bits_to_f32(*reinterpret_cast<const uint16_t*>(smem + kst + ksoff[0]));
-                const float fb = f16_bits_to_f32(*reinterpret_cast<const uint16_t*>(smem + kst + ksoff[0] + 8 * T::KS));
-                sc[0] *= fa; sc[1] *= fa; sc[2] *= fb; sc[3] *= fb;
-            }
-            // q's power of two (and the K tensor scale) back into the fp32 scores
-            sc[0] *= hm0; sc[1] *= hm1; sc[2] *= hm0; sc[3] *= hm1;
-            const bool oka = r < valid, okb = r + 8 < valid;
-            if (!oka) sc[0] = sc[1] = -INFINITY;
-            if (!okb) sc[2] = sc[3] = -INFINITY;
-
-            // ---------- online softmax (log2 domain), heads 2j and 2j+1.  The
-            // running max is raised (with a warp-wide reduction and a rescale of
-            // the accumulators) only when a score exceeds it by more than 2^3;
-            // otherwise weights up to 8 are kept as they are.
-            {
-                const float x0 = fmaxf(sc[0], sc[2]), x1 = fmaxf(sc[1], sc[3]);
-                if (__any_sync(0xffffffffu, (x0 > m0 + 3.f) || (x1 > m1 + 3.f))) {
-                    float y0 = x0, y1 = x1;
-#pragma unroll
-                    for (int m = 4; m < 32; m <<= 1) {
-                        y0 = fmaxf(y0, __shfl_xor_sync(0xffffffffu, y0, m));
-                        y1 = fmaxf(y1, __shfl_xor_sync(0xffffffffu, y1, m));
-                    }
-                    const float n0 = fmaxf(m0, y0), n1 = fmaxf(m1, y1);
-                    const float a0 = (m0 == -INFINITY) ? 0.f : fast_exp2(m0 - n0);
-                    const float a1 = (m1 == -INFINITY) ? 0.f : fast_exp2(m1 - n1);
-#pragma unroll
-                    for (int u = 0; u < T::DTILES / 2; u++) {
-                        o[u][0] *= a0; o[u][1] *= a1; o[u][2] *= a0; o[u][3] *= a1;
-                    }
-                    l0 *= a0;
-                    l1 *= a1;
-                    m0 = n0;
-                    m1 = n1;
-                }
-            }
-            const float r0 = (m0 == -INFINITY) ? 0.f : m0, r1 = (m1 == -INFINITY) ? 0.f : m1;
-            const float p0 = fast_exp2(sc[0] - r0), p1 = fast_exp2(sc[1] - r1);
-            const float p2 = fast_exp2(sc[2] - r0), p3 = fast_exp2(sc[3] - r1);
-            l0 += p0 + p2;
-            l1 += p1 + p3;
-
-            // ---------- O^T += V^T P^T over this warp's half of head_dim
-            // rows past seq_len hold bytes never written: keep them out of the
-            // product entirely (their P is 0, but 0 x NaN would still be NaN)
-            const bool partial = valid < 16;
-            uint32_t pb0 = 0, pb1 = 0;   // P'^T fragment (B operand)
-            // V scales folded into P': this lane's rows r and r + 8, one per
-            // chunk (INT8, MX) or one per row (FP8 row-256), rows past seq_len 0
-            constexpr int NVS = VFOLD ? (KV == RK_E4M3_ROW256 ? 1 : T::VC_HALF) : 1;
-            float vfa[NVS], vfb[NVS];
-            if constexpr (VFOLD) {
-                float smax = 0.f;
-#pragma unroll
-                for (int c = 0; c < NVS; c++) {
-                    if constexpr (KV == RK_E4M3_MX32) {
-                        vfa[c] = ue8m0_to_f32(smem[vst + vsoff[c]]);
-                        vfb[c] = ue8m0_to_f32(smem[vst + vsoff[c] + 8 * T::VS]);
-                    } else {
-                        vfa[c] = f16_bits_to_f32(*reinterpret_cast<const uint16_t*>(smem + vst + vsoff[c]));
-                        vfb[c] = f16_bits_to_f32(*reinterpret_cast<const uint16_t*>(smem + vst + vsoff[c] + 8 * T::VS));
-                    }
-                    vfa[c] = oka ? vfa[c] : 0.f;
-                    vfb[c] = okb ? vfb[c] : 0.f;
-                    smax = fmaxf(smax, fmaxf(vfa[c], vfb[c]));
-                }
-                if (__any_sync(0xffffffffu, smax > vthr)) {
-                    // raise the reference to the warp's largest scale (an exact power of two)
-                    const int en = exp2_floor(__uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(smax))));
-                    const float f = vthr > 0.f ? pow2i(ve - en) : 1.f;
-#pragma unroll
-                    for (int u = 0; u < T::DTILES / 2; u++) {
-                        o[u][0] *= f; o[u][1] *= f; o[u][2] *= f; o[u][3] *= f;
-                    }
-                    ve = en;
-                    vmul = pow2i(-en);
-                    vthr = pow2i(en + 4);
-                }
-#pragma unroll
-                for (int c = 0; c < NVS; c++) {
-                    vfa[c] *= vmul;
-                    vfb[c] *= vmul;
-                }
-            }
-            if constexpr (KV == RK_E4M3_ROW256) {
-                pb0 = movtrans(pack_f16(p0 * vfa[0], p1 * vfa[0]));
-                pb1 = movtrans(pack_f16(p2 * vfb[0], p3 * vfb[0]));
-            } else if constexpr (!VFOLD) {
-                pb0 = movtrans(pack_f16(p0, p1));
-                pb1 = movtrans(pack_f16(p2, p3));
-            }
-#pragma unroll
-            for (int cl = 0; cl < T::VC_HALF; cl++) {
-                if constexpr (KV == RK_INT8_G64 || KV == RK_E4M3_MX32) {
-                    pb0 = movtrans(pack_f16(p0 * vfa[cl], p1 * vfa[cl]));
-                    pb1 = movtrans(pack_f16(p2 * vfb[cl], p3 * vfb[cl]));
-                }
-                uint32_t xa[2 * T::VCH], xb[2 * T::VCH];
-                slice_f16<KV, T::VNB, T::VCH>(lds_bytes<T::VNB>(smem + vt, voff[cl]), xa);
-                slice_f16<KV, T::VNB, T::VCH>(lds_bytes<T::VNB>(smem + vt, voff[cl] + 8 * T::VC), xb);
-                if constexpr (KV == RK_E2M1_G16) {
-                    const uint32_t sa = f16_splat(dec_e4m3x2_f16x2(smem[vst + vsoff[cl]]));
-                    const uint32_t sb = f16_splat(dec_e4m3x2_f16x2(smem[vst + vsoff[cl] + 8 * T::VS]));
-#pragma unroll
-                    for (int e = 0; e < 2 * T::VCH; e++) {
-                        xa[e] = hmul2(xa[e], sa);
-                        xb[e] = hmul2(xb[e], sb);
-                    }
-                }
-                if (partial) {
-#pragma unroll
-                    for (int e = 0; e < 2 * T::VCH; e++) {
-                        xa[e] = oka ? xa[e] : 0u;
-                        xb[e] = okb ? xb[e] : 0u;
-                    }
-                }
-#pragma unroll
-                for (int u = 0; u < T::VCH; u++) {
-                    const uint32_t a[4] = {movtrans(xa[2 * u]), movtrans(xa[2 * u + 1]), movtrans(xb[2 * u]),
-                                           movtrans(xb[2 * u + 1])};
-                    mma_f16(o[cl * T::VCH + u], a, pb0, pb1);
-                }
+            s += ngrp;
+            while (s >= NS) {
+                s -= NS;
+                ph ^= 1u;
             }
         }
 
-        // ---- release stage s; the last warp to release it refills it
-        __syncwarp();
-        if (lane == 0) {
-            __threadfence_block();
-            const int old = atomicAdd(&rel[s], 1);
-            if (old == kDecThreads / 32 - 1) {
-                rel[s] = 0;
-                __threadfence_block();
-                const int k = prod->issued;
-                if (k < n && !*abort_flag) issue(s, (k < p.pid_cap) ? pids[k] : page_id(w0 + k));
-            }
-        }
-
-        const bool seg_end = (i == n - 1) || (cc.span == cc.nspans - 1);
-        if (seg_end) {
-            // ---- merge the warps: max, rescaled sums, rescaled outputs.  The two
-            // warps of a pair hold the same (m, l); the half-0 warp reports them.
+        // ---- segment end: merge the warps -- max, rescaled sums, rescaled
+        // outputs.  Every warp holds a state for the segment (a warp that saw no
+        // token of it has m = -inf, l = 0, o = 0).
 #pragma unroll
-            for (int m = 4; m < 32; m <<= 1) {
-                l0 += __shfl_xor_sync(0xffffffffu, l0, m);
-                l1 += __shfl_xor_sync(0xffffffffu, l1, m);
-            }
-            __syncthreads();   // all tiles of the segment done; osm free
-            for (int k = tid; k < 2 * kOsmStride<D>; k += kDecThreads)
-                reinterpret_cast<float4*>(osm)[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (hf == 0 && r == 0) {
-                wml[tw * 16 + 2 * j] = m0;
-                wml[tw * 16 + 2 * j + 1] = m1;
-                wml[tw * 16 + 8 + 2 * j] = l0;
-                wml[tw * 16 + 8 + 2 * j + 1] = l1;
-            }
-            __syncthreads();
+        for (int m = 4; m < 32; m <<= 1) {
+            l0 += __shfl_xor_sync(0xffffffffu, l0, m);
+            l1 += __shfl_xor_sync(0xffffffffu, l1, m);
+        }
+        if (r == 0) {
+            wml[warp * 16 + 2 * j] = m0;
+            wml[warp * 16 + 2 * j + 1] = m1;
+            wml[warp * 16 + 8 + 2 * j] = l0;
+            wml[warp * 16 + 8 + 2 * j + 1] = l1;
+        }
+        __syncthreads();   // every warp's units of the segment done; osm free
+        {
             float M0 = -INFINITY, M1 = -INFINITY;
 #pragma unroll
-            for (int w = 0; w < 4; w++) {
+            for (int w = 0; w < 8; w++) {
                 M0 = fmaxf(M0, wml[w * 16 + 2 * j]);
                 M1 = fmaxf(M1, wml[w * 16 + 2 * j + 1]);
             }
@@ -1028,77 +1027,100 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
             const float f1 = (m1 == -INFINITY) ? 0.f : exp2f(m1 - M1) * vu;
             if (tid < 8) {
                 float M = -INFINITY, Ls = 0.f;
-                for (int w = 0; w < 4; w++) M = fmaxf(M, wml[w * 16 + tid]);
-                for (int w = 0; w < 4; w++) {
-                    float mw = wml[w * 16 + tid];
+                for (int w = 0; w < 8; w++) M = fmaxf(M, wml[w * 16 + tid]);
+                for (int w = 0; w < 8; w++) {
+                    const float mw = wml[w * 16 + tid];
                     if (mw != -INFINITY) Ls += exp2f(mw - M) * wml[w * 16 + 8 + tid];
                 }
                 fin[tid] = M;
                 fin[8 + tid] = Ls;
             }
-            {
-                // this lane's outputs: heads 2j, 2j+1; dims (relative to its half)
-                // VCW*(ul/VCH) + 4*(ul%VCH) + [0 | 2] + lane part
-                float* pa = osm + (2 * j) * kOsmStride<D> + hf * (D / 2) + 4 * T::VCH * (r >> 1) + (r & 1);
-                float* pb = pa + kOsmStride<D>;
-#pragma unroll 1
-                for (int w = 0; w < 4; w++) {
-                    if (tw == w) {   // both halves write disjoint head_dim ranges
+            // eight rounds: in round q warp w adds d-tile chunk (w + q) % 8 of its
+            // output into the combine buffer (round 0 stores), so all warps work in
+            // every round on disjoint chunks; the order of the sum is fixed.  A
+            // lane's values: heads 2j, 2j+1; dims VCW*(u/VCH) + 4*(u%VCH) + [0 | 2]
+            // + its row part (u the d-tile).  The chunk is picked by a switch so
+            // that o is indexed statically and stays in registers.
+            float* pa = osm + (2 * j) * kOsmStride<D> + 4 * T::VCH * (r >> 1) + (r & 1);
+            float* pb = pa + kOsmStride<D>;
+            constexpr int DT8 = T::DTILES / 8;
+            // d-tiles u of chunk ch (a static index into o for each case)
+            auto add_chunk = [&](auto chc, bool first) {
+                constexpr int ch = decltype(chc)::value;
 #pragma unroll
-                        for (int ul = 0; ul < T::DTILES / 2; ul++) {
-                            const int d = T::VCW * (ul / T::VCH) + 4 * (ul % T::VCH);
-                            pa[d] += o[ul][0] * f0; pb[d] += o[ul][1] * f1;
-                            pa[d + 2] += o[ul][2] * f0; pb[d + 2] += o[ul][3] * f1;
-                        }
+                for (int z = 0; z < DT8; z++) {
+                    const int u2 = ch * DT8 + z;
+                    const int d = T::VCW * (u2 / T::VCH) + 4 * (u2 % T::VCH);
+                    if (first) {
+                        pa[d] = o[u2][0] * f0; pb[d] = o[u2][1] * f1;
+                        pa[d + 2] = o[u2][2] * f0; pb[d + 2] = o[u2][3] * f1;
+                    } else {
+                        pa[d] += o[u2][0] * f0; pb[d] += o[u2][1] * f1;
+                        pa[d + 2] += o[u2][2] * f0; pb[d + 2] += o[u2][3] * f1;
                     }
-                    __syncthreads();
                 }
+            };
+#pragma unroll 1
+            for (int q = 0; q < 8; q++) {
+                const bool first = q == 0;
+                switch ((warp + q) & 7) {
+                case 0: add_chunk(std::integral_constant<int, 0>{}, first); break;
+                case 1: add_chunk(std::integral_constant<int, 1>{}, first); break;
+                case 2: add_chunk(std::integral_constant<int, 2>{}, first); break;
+                case 3: add_chunk(std::integral_constant<int, 3>{}, first); break;
+                case 4: add_chunk(std::integral_constant<int, 4>{}, first); break;
+                case 5: add_chunk(std::integral_constant<int, 5>{}, first); break;
+                case 6: add_chunk(std::integral_constant<int, 6>{}, first); break;
+                default: add_chunk(std::integral_constant<int, 7>{}, first); break;
+                }
+                __syncthreads();
             }
+        }
 
-            // ---- a whole segment is normalised and stored here; a segment cut by
-            // a range boundary leaves its unnormalised output as this CTA's partial
-            // (rotated back already: the Hadamard is linear, so merging commutes
-            // with it) for the merge after the grid barrier.
-            const int64_t seg_w0 = (int64_t)pref[b] * HH + (int64_t)cc.hh * cc.nspans;
-            const bool whole = (seg_w0 >= w0) && (seg_w0 + cc.nspans <= w1);
+        // ---- a whole segment is normalised and stored here; a segment cut by
+        // a range boundary leaves its unnormalised output as this CTA's partial
+        // (rotated back already: the Hadamard is linear, so merging commutes
+        // with it) for the merge after the grid barrier.
+        {
+            const int64_t seg_w0 = (int64_t)pref[b] * HH + (int64_t)cc.hh * nspans;
+            const bool whole = (seg_w0 >= w0) && (seg_w0 + nspans <= w1);
             float* part = p.partials + ((int64_t)blockIdx.x * 2 + (seg_first ? 0 : 1)) * (16 + 8 * D);
             if (!whole && tid < 16) part[tid] = fin[tid];
-            {
-                const int nh = warp;   // warp w finishes head w of the block
-                const int gq = hb * 8 + nh;
-                if (gq < p.G) {
-                    const float Ls = fin[8 + nh];
-                    const float inv = whole ? ((Ls > 0.f) ? p.o_mult / Ls : 0.f) : 1.f;
-                    float x[8];
+            const int nh = warp;   // warp w finishes head w of the block
+            const int gq = hb * 8 + nh;
+            if (gq < p.G) {
+                const float Ls = fin[8 + nh];
+                const float inv = whole ? ((Ls > 0.f) ? p.o_mult / Ls : 0.f) : 1.f;
+                float x[8];
 #pragma unroll
-                    for (int e = 0; e < T::EPL; e++) x[e] = osm[nh * kOsmStride<D> + lane * T::EPL + e] * inv;
-                    if constexpr (D == 256) {
-                        if (p.rot_v) {
-                            Row8 y;
+                for (int e = 0; e < T::EPL; e++) x[e] = osm[nh * kOsmStride<D> + lane * T::EPL + e] * inv;
+                if constexpr (D == 256) {
+                    if (p.rot_v) {
+                        Row8 y;
 #pragma unroll
-                            for (int e = 0; e < 8; e++) y.v[e] = x[e];
-                            y = fwht256_row(y, lane);
+                        for (int e = 0; e < 8; e++) y.v[e] = x[e];
+                        y = fwht256_row(y, lane);
 #pragma unroll
-                            for (int e = 0; e < 8; e++) x[e] = y.v[e];
-                        }
-                    }
-                    if (!whole) {
-                        float* dst = part + 16 + nh * D + lane * T::EPL;
-#pragma unroll
-                        for (int e = 0; e < T::EPL; e += 4)
-                            *reinterpret_cast<float4*>(dst + e) = make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]);
-                    } else {
-                        const int64_t ob = ((int64_t)b * p.Hq + h * p.G + gq) * D + lane * T::EPL;
-                        store_out<T::EPL>(p.out, p.out_fp32, ob, x);
+                        for (int e = 0; e < 8; e++) x[e] = y.v[e];
                     }
                 }
+                if (!whole) {
+                    float* dst = part + 16 + nh * D + lane * T::EPL;
+#pragma unroll
+                    for (int e = 0; e < T::EPL; e += 4)
+                        *reinterpret_cast<float4*>(dst + e) = make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]);
+                } else {
+                    const int64_t ob = ((int64_t)b * p.Hq + h * p.G + gq) * D + lane * T::EPL;
+                    store_out<T::EPL>(p.out, p.out_fp32, ob, x);
+                }
             }
-            __syncthreads();   // osm and fin are free again
         }
-        cursor_next(cc, pref, B, HH, HB);
-        if (++s == NS) {
-            s = 0;
-            ph ^= 1u;
+        __syncthreads();   // osm, fin and qst are free again
+
+        i += seg_n;
+        if (i < n) {   // to the next segment's first unit
+            cc.span = nspans - 1;
+            cursor_next(cc, pref, B, HH, HB);
         }
     }
 
@@ -1106,11 +1128,10 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
     if (*abort_flag) {
         if (tid == 0) {
             atomicOr(p.status, kStatusWaitTimeout);
-            // wait (bounded) for the copies still in flight: the last NS issued
+            // wait (bounded) for the copies still in flight: the last one issued into each stage
             int dummy = 0;
-            const int k0 = prod->issued > NS ? prod->issued - NS : 0;
-            for (int k = k0; k < prod->issued; k++)
-                (void)mbar_wait(smem_u32(&bars[k % NS]), (uint32_t)((k / NS) & 1), &dummy);
+            for (int s2 = 0; s2 < NS; s2++)
+                if (iss[s2] > 0) (void)mbar_wait(smem_u32(&bars[s2]), (uint32_t)((iss[s2] - 1) & 1), &dummy);
         }
         __syncthreads();
     }
@@ -1170,9 +1191,9 @@ bool decode_supported(int fmt, int D) {
 
 static size_t fixed_smem(int D, int B, int pid_cap, int qs) {
     const size_t ostr = (size_t)D + 4;   // kOsmStride
-    const size_t osm = 8 * ostr * 4 > 8192 ? 8 * ostr * 4 : 8192;
+    const size_t osm = 8 * ostr * 4;
     const size_t qst = 8 * (size_t)D * 2 * qs;
-    return 8 * kMaxStages + 4 * kMaxStages + 32 + osm + qst + 4 * 16 * 4 + 16 * 4 + 8 * 4 + 16 + 4 * (size_t)(B + 1) +
+    return 8 * kMaxStages + 3 * 4 * kMaxStages + osm + qst + 8 * 16 * 4 + 16 * 4 + 8 * 4 + 16 + 4 * (size_t)(B + 1) +
            4 * (size_t)pid_cap + 128;
 }
 
