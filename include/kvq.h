@@ -144,7 +144,7 @@ size_t kvq_decode_workspace_bytes(const kvq_cache* cache, int32_t batch, int32_t
  * For rotated K the kernel rotates q by the same Hadamard-256 (q.k is unchanged
  * because the rotation is orthonormal); for rotated V it rotates the output
  * back.  Page ids out of range are replaced by page 0 and recorded in the
- * device status word. */
+ * device status word.  Limit: num_pages * n_kv_heads < 2^30 (KVQ_ERR_SHAPE). */
 int kvq_decode_attention(kvq_cache* cache, int32_t layer, const void* q, int32_t n_q_heads,
                          const int32_t* block_table, int32_t max_pages_per_seq,
                          const int32_t* seq_lens, int32_t batch, int32_t max_seq_len,

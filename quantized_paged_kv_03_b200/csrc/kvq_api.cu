@@ -208,6 +208,8 @@ int kvq::decode_setup(kvq_cache* cache, int32_t layer, const void* k_new, const 
     if ((int64_t)max_pages_per_seq * cache->L.P < max_seq_len) return KVQ_ERR_SHAPE;
     if (((uintptr_t)q & 15) || ((uintptr_t)out & 15)) return KVQ_ERR_ARG;
     if (!(softmax_scale >= 0.f) || !isfinite(softmax_scale)) return KVQ_ERR_ARG;
+    // the kernel names a page slab by a 30-bit index (page * n_kv_heads + kv-head)
+    if ((int64_t)cache->L.num_pages * cache->L.H >= ((int64_t)1 << 30)) return KVQ_ERR_SHAPE;
     DecodeParams& p = *pp;
     p.L = cache->L;
     p.slabs = layer_slabs(cache, layer);
@@ -253,6 +255,7 @@ int kvq::decode_launch(DecodeParams* p, const DecodePlan& plan, void* workspace,
     decode_workspace_zero_region(p->L, p->B, p->HB, plan.grid, &zoff, &zbytes);
     p->partials = (float*)workspace;
     p->barrier = (unsigned*)((uint8_t*)workspace + zoff);
+    p->seg_count = p->barrier + 64;   // after the barrier's 256-byte block
     return cuda_status(launch_decode(*p, plan, stream));
 }
 

@@ -49,6 +49,9 @@ template <int D>
 constexpr int kOsmStride = D + 4;
 constexpr int kMaxStages = 8;
 constexpr int kMaxBatch = 4096;
+// A cut segment with at most this many parts is merged by the CTA that
+// completes it; one with more is merged by all of its CTAs after a grid barrier.
+constexpr int kFewParts = 16;
 constexpr long kWaitPolls = 1l << 22;
 
 // ------------------------------------------------------------ PTX helpers
@@ -309,9 +312,10 @@ __device__ __forceinline__ void store_out(void* out, int out_fp32, int64_t ob, c
 
 // Grid-wide barrier of the G co-resident CTAs (cooperative launch).  Arrival
 // counter + generation word in the workspace; the last arriver resets the
-// counter, so it is zero again after every launch.  The wait is bounded: on
+// counter, so it is zero again after every launch.  Every CTA arrives; only a
+// CTA that passes `wait` waits for the others.  The wait is bounded: on
 // timeout the CTA records it and returns false.
-__device__ __forceinline__ bool grid_barrier(unsigned* bar, unsigned G, int* flag_smem) {
+__device__ __forceinline__ bool grid_barrier(unsigned* bar, unsigned G, int* flag_smem, bool wait) {
     __syncthreads();
     if (threadIdx.x == 0) {
         volatile unsigned* vgen = bar + 1;
@@ -323,7 +327,7 @@ __device__ __forceinline__ bool grid_barrier(unsigned* bar, unsigned G, int* fla
             atomicExch(bar, 0u);
             __threadfence();
             atomicAdd(bar + 1, 1u);
-        } else {
+        } else if (wait) {
             long it = 0;
             while (*vgen == gen) {
                 __nanosleep(64);
@@ -340,23 +344,22 @@ __device__ __forceinline__ bool grid_barrier(unsigned* bar, unsigned G, int* fla
     return *flag_smem != 0;
 }
 
-// Merge share `j` of the partials of one cut segment (CTAs i_first..i_last
-// each left (max, sum, unnormalised output) for up to 8 query heads): this CTA
-// produces float4 outputs [o0, o1) of the segment's gv x D/4.  One pass: each
+// Merge share j of nshares of the partials of one cut segment (CTAs
+// i_first..i_last each left (max, sum, unnormalised output) for up to 8 query
+// heads): this CTA produces float4 outputs [o0, o1) of the segment's gv x D/4.  One pass: each
 // output's threads fold the parts in with a running (max, sum, output) -- the
 // log-sum-exp merge -- then combine their folds by shuffles; no block barrier.
-constexpr int kMergeBatch = 2;
+constexpr int kMergeBatch = 8;   // parts whose loads are in flight together
 
 template <int D>
 __device__ __forceinline__ void merge_segment(const float* partials, void* out, int out_fp32, float o_mult, int Hq,
                                            int Gq, int b, int h, int hb, int64_t seg_w0, int i_first, int i_last,
-                                           Partition part) {
+                                           Partition part, int j, int nshares) {
     const int tid = threadIdx.x;
     const int P = i_last - i_first + 1;
-    const int j = (int)blockIdx.x - i_first;
     const int gv = min(8, Gq - hb * 8);
     const int NU = gv * (D / 4);
-    const int o0 = (int)((int64_t)j * NU / P), o1 = (int)((int64_t)(j + 1) * NU / P);
+    const int o0 = (int)((int64_t)j * NU / nshares), o1 = (int)((int64_t)(j + 1) * NU / nshares);
     const int no = o1 - o0;
     if (no <= 0) return;
     // The segment is the first of every part's range except possibly the first
@@ -615,16 +618,40 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
             tagv[s] = -1;
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        // the first stages' block-table entries, all loads in flight together
         Cursor c;
         cursor_locate(c, w0, pref, B, HH, HB);
+        int raw[kMaxStages];
+        uint32_t hspan[kMaxStages];
 #pragma unroll
         for (int s = 0; s < kMaxStages; s++) {
             if (s < NS && s < n) {
-                pids[s] = (int)unit_word(c);
+                raw[s] = __ldg(p.block_table + (int64_t)c.b * p.max_pages + (c.span >> U.lg_up));
+                hspan[s] = ((uint32_t)c.h << 2) | ((uint32_t)c.span & span_mask);
                 cursor_next(c, pref, B, HH, HB);
             }
         }
+#pragma unroll
+        for (int s = 0; s < kMaxStages; s++)
+            if (s < NS && s < n)
+                pids[s] = (int)(((uint32_t)(checked(raw[s]) * H) << 2) + hspan[s]);
         for (int s = 0; s < NS && s < n; s++) issue(s, s);
+    }
+    {
+        // the q rows of the range's first segments, towards L2 ahead of their
+        // segment starts (rows of one 8-head block are contiguous)
+        Cursor c;
+        cursor_locate(c, w0, pref, B, HH, HB);
+        int64_t w = w0;
+        for (int k = 0; k < 8 && w < w1; k++) {
+            const int gq0 = c.hb * 8, rows = min(8, p.G - gq0);
+            const uint16_t* q0 = p.q + ((int64_t)c.b * p.Hq + (int64_t)c.h * p.G + gq0) * D;
+            if (tid < rows * D * 2 / 128)
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(q0 + tid * 64));
+            w += c.nspans - c.span;
+            c.span = c.nspans - 1;
+            cursor_next(c, pref, B, HH, HB);
+        }
     }
     for (int k = NS + tid; k < n && k < p.pid_cap; k += kDecThreads) {
         Cursor c;
@@ -1136,15 +1163,19 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
         __syncthreads();
     }
 
-    // ---- merge the cut segments, spread over every CTA that holds a part
+    // ---- merge the cut segments.  A segment cut into at most kFewParts parts
+    // is merged by the CTA that completes it -- the last of its parts to count
+    // itself in -- so no CTA waits on another; a segment with more parts is
+    // merged after a grid barrier, a share by every CTA that holds a part.
+    // Every CTA arrives at the barrier; only those with such a share wait.
+    // (A CTA whose cost share holds no unit still arrives: the barrier counts G.)
     if (G > 1) {
-        if (!grid_barrier(p.barrier, (unsigned)G, &flags[2])) {
-            if (tid == 0) atomicOr(p.status, kStatusWaitTimeout);
-            return;
-        }
         Cursor c0, c1;
-        cursor_locate(c0, w0, pref, B, HH, HB);
-        cursor_locate(c1, w1 - 1, pref, B, HH, HB);
+        if (n > 0) {
+            cursor_locate(c0, w0, pref, B, HH, HB);
+            cursor_locate(c1, w1 - 1, pref, B, HH, HB);
+        }
+        bool wait = false;
         for (int k = 0; k < (n > 0 ? 2 : 0); k++) {
             const Cursor& c = k == 0 ? c0 : c1;
             if (k == 1 && c1.b == c0.b && c1.hh == c0.hh) break;
@@ -1152,8 +1183,44 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
             if (seg_w0 >= w0 && seg_w0 + c.nspans <= w1) continue;     // whole: already stored
             const int i_first = part.owner(c.b, c.hh, 0);
             const int i_last = part.owner(c.b, c.hh, c.nspans - 1);
-            merge_segment<D>(p.partials, p.out, p.out_fp32, p.o_mult, p.Hq, p.G, c.b, c.h, c.hb, seg_w0, i_first,
-                             i_last, part);
+            if (i_last - i_first + 1 > kFewParts) {
+                wait = true;
+                continue;
+            }
+            // count this part in; the last to arrive merges the segment and
+            // clears its counter for the next call (counters are indexed by the
+            // CTA holding the segment's end, which ends at most one cut segment)
+            __syncthreads();   // this CTA's partial is written
+            if (tid == 0) {
+                __threadfence();
+                const unsigned old = atomicAdd(&p.seg_count[i_last], 1u);
+                flags[1] = (old == (unsigned)(i_last - i_first));
+                if (flags[1]) {
+                    p.seg_count[i_last] = 0u;
+                    __threadfence();
+                }
+            }
+            __syncthreads();
+            if (flags[1])
+                merge_segment<D>(p.partials, p.out, p.out_fp32, p.o_mult, p.Hq, p.G, c.b, c.h, c.hb, seg_w0, i_first,
+                                 i_last, part, 0, 1);
+        }
+        if (!grid_barrier(p.barrier, (unsigned)G, &flags[2], wait)) {
+            if (tid == 0) atomicOr(p.status, kStatusWaitTimeout);
+            return;
+        }
+        if (wait) {
+            for (int k = 0; k < 2; k++) {   // (wait is set only when n > 0)
+                const Cursor& c = k == 0 ? c0 : c1;
+                if (k == 1 && c1.b == c0.b && c1.hh == c0.hh) break;
+                const int64_t seg_w0 = (int64_t)pref[c.b] * HH + (int64_t)c.hh * c.nspans;
+                if (seg_w0 >= w0 && seg_w0 + c.nspans <= w1) continue;
+                const int i_first = part.owner(c.b, c.hh, 0);
+                const int i_last = part.owner(c.b, c.hh, c.nspans - 1);
+                if (i_last - i_first + 1 <= kFewParts) continue;
+                merge_segment<D>(p.partials, p.out, p.out_fp32, p.o_mult, p.Hq, p.G, c.b, c.h, c.hb, seg_w0, i_first,
+                                 i_last, part, (int)blockIdx.x - i_first, i_last - i_first + 1);
+            }
         }
     }
 }
@@ -1260,17 +1327,21 @@ static size_t partial_bytes(const Layout& L, int grid) {
     return (((size_t)grid * 2 * (16 + 8 * (size_t)L.D) * sizeof(float)) + 255) & ~(size_t)255;
 }
 
+// Zeroed region: the grid barrier's two words, then one counter per CTA (the
+// parts of the cut segment that ends in that CTA's range).
+static size_t zero_bytes(int grid) { return (256 + 4 * (size_t)grid + 255) & ~(size_t)255; }
+
 size_t decode_workspace_bytes(const Layout& L, int B, int HB, int grid) {
     (void)B;
     (void)HB;
-    return partial_bytes(L, grid) + 256;
+    return partial_bytes(L, grid) + zero_bytes(grid);
 }
 
 void decode_workspace_zero_region(const Layout& L, int B, int HB, int grid, size_t* offset, size_t* bytes) {
     (void)B;
     (void)HB;
     *offset = partial_bytes(L, grid);
-    *bytes = 256;
+    *bytes = zero_bytes(grid);
 }
 
 cudaError_t launch_decode(const DecodeParams& p, const DecodePlan& plan, cudaStream_t s) {

@@ -74,6 +74,7 @@ struct DecodeParams {
     long wait_polls;             // polls of a pipeline wait before it gives up
     float* partials;             // [gridDim.x][2][16 + 8 * D]: (max, sum, output) of cut segments
     unsigned* barrier;           // grid barrier: [0] arrivals (zero between calls), [1] generation
+    unsigned* seg_count;         // [gridDim.x] parts counted in of the cut segment ending in each CTA's range
     uint32_t* status;
     int stages;                  // pipeline depth (page slabs in shared memory)
     int pid_cap;                 // page ids of a CTA's range preloaded into shared memory
