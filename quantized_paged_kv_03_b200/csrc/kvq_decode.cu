@@ -608,34 +608,24 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
         __threadfence_block();
         tagv[s] = k;
     };
-    // thread 0 starts the ring with its own block-table reads (all in flight at
-    // once) while the other threads preload the range's unit sources
-    if (tid == 0) {
-        for (int s = 0; s < NS; s++) {
-            mbar_init(smem_u32(&bars[s]), 1);
-            rel[s] = 0;
-            iss[s] = 0;
-            tagv[s] = -1;
+    // warp 0 starts the ring, lane s with stage s: its own cursor, block-table
+    // read and copy, so that the first stages' latencies overlap, while the
+    // other warps preload the range's unit sources
+    if (warp == 0) {
+        if (lane < NS) {
+            mbar_init(smem_u32(&bars[lane]), 1);
+            rel[lane] = 0;
+            iss[lane] = 0;
+            tagv[lane] = -1;
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        // the first stages' block-table entries, all loads in flight together
-        Cursor c;
-        cursor_locate(c, w0, pref, B, HH, HB);
-        int raw[kMaxStages];
-        uint32_t hspan[kMaxStages];
-#pragma unroll
-        for (int s = 0; s < kMaxStages; s++) {
-            if (s < NS && s < n) {
-                raw[s] = __ldg(p.block_table + (int64_t)c.b * p.max_pages + (c.span >> U.lg_up));
-                hspan[s] = ((uint32_t)c.h << 2) | ((uint32_t)c.span & span_mask);
-                cursor_next(c, pref, B, HH, HB);
-            }
+        __syncwarp();
+        if (lane < NS && lane < n) {
+            Cursor c;
+            cursor_locate(c, w0 + lane, pref, B, HH, HB);
+            pids[lane] = (int)unit_word(c);
+            issue(lane, lane);
         }
-#pragma unroll
-        for (int s = 0; s < kMaxStages; s++)
-            if (s < NS && s < n)
-                pids[s] = (int)(((uint32_t)(checked(raw[s]) * H) << 2) + hspan[s]);
-        for (int s = 0; s < NS && s < n; s++) issue(s, s);
     }
     {
         // the q rows of the range's first segments, towards L2 ahead of their
@@ -1349,8 +1339,10 @@ cudaError_t launch_decode(const DecodeParams& p, const DecodePlan& plan, cudaStr
     if (!k) return cudaErrorInvalidValue;
     DecodeParams q = p;
     q.U = make_span(p.L, plan.lg_up);
-    // cost of a segment's start and end in units (about four 64-token units)
-    q.seg_cost = q.U.sp >= 256 ? 1 : 256 / q.U.sp;
+    // cost of a segment's start, end and merge in units: about 512 tokens of
+    // streaming (measured on B200 over the five decode workloads; 256 and 768
+    // were both slower)
+    q.seg_cost = q.U.sp >= 256 ? 2 : 512 / q.U.sp;
     void* args[] = {&q};
     // cooperative: the merge after the grid barrier needs every CTA resident
     return cudaLaunchCooperativeKernel(k, dim3(plan.grid), dim3(plan.threads), args, plan.smem, s);
