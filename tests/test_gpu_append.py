@@ -130,3 +130,98 @@ def test_zero_rows_and_tiny_rows():
         got = [t.cpu().numpy() for t in c.read_rows(0, dev(slots))]
         for g, want in zip(got, (oc.kc, oc.ks, oc.vc, oc.vs)):
             assert np.array_equal(g, want[slots]), fmt
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("D", [256, 128])
+def test_int8_codes_on_rounding_ties(D):
+    """INT8 rows whose quotients value / scale land exactly on half-integers
+    (each 64-group's amax is 127 x 2^j, so its fp16 scale is 2^j, and the other
+    values are (k + 1/2) x 2^j): the codes must equal the oracle's, which
+    rounds the correctly rounded quotient half to even."""
+    r = np.random.default_rng(11)
+    P, n = 64, 48
+    rows = []
+    for t in range(n):
+        j = int(r.integers(-20, 12))
+        k = r.integers(0, 127, size=D).astype(np.float64)
+        x = (k + 0.5) * r.choice([-1.0, 1.0], size=D)
+        x[(np.arange(D) % 64) == (t % 64)] = 127.0          # one amax per group
+        rows.append(x * 2.0 ** j)
+    x = np.array(rows, np.float32)[:, None, :]
+    bits = I.bf16_bits(x)
+    assert np.array_equal(I.bf16_to_f32(bits), x)             # every value is a bf16 value
+    slots = np.arange(n, dtype=np.int64) + P
+    c = K.KVCache("int8_g64", D, 1, P, 2, flags=K.FLAG_NO_ROTATE)
+    c.append(0, bf16_dev(bits), bf16_dev(bits), dev(slots))
+    oc = O.PagedCache(K.FORMATS["int8_g64"], D, 1, P, 2, flags=K.FLAG_NO_ROTATE)
+    oc.append(bits, bits, slots)
+    got = [t.cpu().numpy() for t in c.read_rows(0, dev(slots))]
+    for g, want in zip(got, (oc.kc, oc.ks, oc.vc, oc.vs)):
+        assert np.array_equal(g, want[slots])
+    codes = oc.kc[slots].view(np.int8).astype(np.int64)
+    assert (np.abs(codes) % 2 == 0).sum() > 0.4 * codes.size   # ties went to even codes
+
+
+def e4m3_midpoints():
+    """Every rounding boundary of E4M3 up to 448, subnormal range included:
+    midpoints of consecutive grid values, as float64."""
+    g = [j * 2.0 ** -9 for j in range(8)]                                  # subnormals
+    g += [(1 + m / 8) * 2.0 ** e for e in range(-6, 9) for m in range(8)]  # normals
+    g = np.array(sorted(v for v in g if v <= 448.0))
+    return (g[1:] + g[:-1]) / 2
+
+
+E2M1_MIDPOINTS = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("fmt", ["nvfp4_g16", "fp8_row256", "fp8_tensor", "k8v4"])
+def test_codes_on_grid_rounding_boundaries(fmt):
+    """Rows whose quotients value / scale land exactly on the encoder's rounding
+    boundaries (midpoints of the E2M1 or E4M3 grid, E4M3's subnormal range
+    included), or one bf16 step beside them: every code must equal the
+    oracle's, which rounds the correctly rounded quotient to nearest even.
+    Rotation is off so that the quotients are the constructed ones."""
+    r = np.random.default_rng(17)
+    D, P, n = 256, 64, 40
+    mids = {"fp8_row256": e4m3_midpoints(), "fp8_tensor": e4m3_midpoints(), "nvfp4_g16": E2M1_MIDPOINTS}
+    top = {"fp8_row256": 448.0, "fp8_tensor": 448.0, "nvfp4_g16": 6.0}
+    group = {"fp8_row256": 256, "fp8_tensor": 256, "nvfp4_g16": 16}
+
+    def rows(kind, pow2):
+        out = []
+        for t in range(n):
+            j = pow2[t]
+            m = r.choice(mids[kind], size=D)
+            m = m * r.choice([-1.0, 1.0], size=D)
+            beside = r.random(D) < 0.3                           # one bf16 step off the boundary
+            m = np.where(beside, m * (1 + r.choice([-1.0, 1.0], size=D) * 2.0 ** -7), m)
+            m[(np.arange(D) % group[kind]) == (t % group[kind])] = top[kind]   # each group's amax
+            out.append(m * 2.0 ** j)
+        x = np.array(out, np.float32)[:, None, :]
+        bits = I.bf16_bits(x)
+        return bits
+
+    if fmt == "k8v4":
+        kb = rows("fp8_row256", r.integers(-12, 8, size=n))
+        vb = rows("nvfp4_g16", r.integers(-9, 8, size=n))
+        scales = None
+    elif fmt == "fp8_tensor":
+        kb = rows(fmt, np.zeros(n, int))
+        vb = rows(fmt, np.full(n, -3))
+        scales = (1.0, 0.125)          # the tensor scales put the quotients on the boundaries
+    else:
+        lo, hi = (-9, 8) if fmt == "nvfp4_g16" else (-12, 8)
+        kb = rows(fmt, r.integers(lo, hi, size=n))
+        vb = rows(fmt, r.integers(lo, hi, size=n))
+        scales = None
+    slots = np.arange(n, dtype=np.int64) + P
+    c = K.KVCache(fmt, D, 1, P, 2, 1, K.FLAG_NO_ROTATE, [scales] if scales else None)
+    c.append(0, bf16_dev(kb), bf16_dev(vb), dev(slots))
+    sk, sv = scales if scales else (1.0, 1.0)
+    oc = O.PagedCache(K.FORMATS[fmt], D, 1, P, 2, K.FLAG_NO_ROTATE, sk, sv)
+    oc.append(kb, vb, slots)
+    got = [t.cpu().numpy() for t in c.read_rows(0, dev(slots))]
+    for g, want, name in zip(got, (oc.kc, oc.ks, oc.vc, oc.vs), ("K codes", "K scales", "V codes", "V scales")):
+        assert np.array_equal(g, want[slots]), name
