@@ -93,6 +93,9 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t phase, volatile
     *abort = 1;
     return false;
 }
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
                  "l"(src), "r"(bytes), "r"(bar)
@@ -149,16 +152,29 @@ __device__ __forceinline__ uint32_t p_off(int r, int c) { return (uint32_t)((c >
 // `smul` = 2^-e, e the sequence's scale exponent (sequence_scale_exps): INT8,
 // E4M3 row-256 and MX scales enter as scale x 2^-e, so every dequantised value
 // lies below 2 x the largest code, inside fp16's range.
+template <int KIND>
+__device__ __forceinline__ uint32_t chunk_scale_bits(const uint8_t* srow, int j) {
+    if constexpr (kind_bits(KIND) == 4) {
+        return (uint32_t)srow[2 * j] | ((uint32_t)srow[2 * j + 1] << 8);   // the chunk's two UE4M3 scales
+    } else if constexpr (KIND == RK_INT8_G64 || KIND == RK_E4M3_ROW256) {
+        const int g = j * 16 / kind_group(KIND);
+        return (uint32_t)srow[2 * g] | ((uint32_t)srow[2 * g + 1] << 8);   // fp16 scale of the chunk's group
+    } else if constexpr (KIND == RK_E4M3_MX32) {
+        return srow[j * 16 / 32];                                          // UE8M0 scale of the chunk's group
+    } else {
+        return 0u;
+    }
+}
+
 template <int KIND, int D>
-__device__ __forceinline__ void dequant_chunk(const uint4 w, const uint8_t* srow, int j, uint8_t* tile, int t, int T,
+__device__ __forceinline__ void dequant_chunk(const uint4 w, uint32_t sbits, int j, uint8_t* tile, int t, int T,
                                               float smul) {
-    constexpr int SB = kind_scale_bytes(KIND);
     const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
     if constexpr (kind_bits(KIND) == 16) {
         *reinterpret_cast<uint4*>(tile + kv_off(t, j * 8, T)) = w;   // bf16 keys / fp16 values: the stored bits
     } else if constexpr (kind_bits(KIND) == 4) {
         // 32 E2M1 codes (two groups of 16, UE4M3 scales): code x scale is exact in fp16
-        const uint32_t sc = dec_e4m3x2_f16x2((uint32_t)srow[2 * j] | ((uint32_t)srow[2 * j + 1] << 8));
+        const uint32_t sc = dec_e4m3x2_f16x2(sbits);
         const uint32_t s0 = splat16(sc), s1 = splat16(sc >> 16);
         uint32_t h[16];
 #pragma unroll
@@ -180,14 +196,13 @@ __device__ __forceinline__ void dequant_chunk(const uint4 w, const uint8_t* srow
         }
         if constexpr (KIND == RK_INT8_G64 || KIND == RK_E4M3_ROW256) {
             // fp16 scale: one nearest-even rounding of code x scale
-            const int g = j * 16 / kind_group(KIND);
-            const float sf = f16_bits_to_f32((uint32_t)srow[SB * g] | ((uint32_t)srow[SB * g + 1] << 8)) * smul;
+            const float sf = f16_bits_to_f32(sbits) * smul;
             const uint32_t sc = splat16(__half_as_ushort(__float2half_rn(sf)));
 #pragma unroll
             for (int i = 0; i < 8; i++) h[i] = mul_f16x2(h[i], sc);
         } else if constexpr (KIND == RK_E4M3_MX32) {
             // UE8M0 scale 2^(e-127): applied in fp32 (exact), then to fp16
-            const float sc = ue8m0_to_f32(srow[j * 16 / 32]) * smul;
+            const float sc = ue8m0_to_f32(sbits) * smul;
 #pragma unroll
             for (int i = 0; i < 8; i++) {
                 const float2 f = f16x2_to_f32(h[i]);
@@ -234,7 +249,7 @@ __device__ __forceinline__ void dequant_tile(const uint8_t* codes, const uint8_t
             for (int e = 0; e < EPC / 8; e++)
                 *reinterpret_cast<uint4*>(tile + kv_off(t, j * EPC + 8 * e, T)) = make_uint4(0, 0, 0, 0);
         } else {
-            dequant_chunk<KIND, D>(w[i], scales + t * SB, j, tile, t, T, smul);
+            dequant_chunk<KIND, D>(w[i], chunk_scale_bits<KIND>(scales + t * SB, j), j, tile, t, T, smul);
         }
     }
 }
@@ -283,10 +298,10 @@ __device__ __forceinline__ int scale_exp_of_bits(uint32_t mx) {
 // every value lies below 2 x the largest code, and the 2^e goes back in fp32.
 // One pass over the scale rows (16 bytes per token for INT8 at head_dim 256),
 // once per CTA, while the ring's first copies are in flight.
-template <int KK, int KV, int D>
+template <int KK, int KV, int D, int NT = kPrefillThreads>
 __device__ void sequence_scale_exps(const PrefillParams& p, int b, int hh, int Ls, uint32_t* red, int* ek, int* ev) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    constexpr int NW = kPrefillThreads / 32;
+    constexpr int NW = NT / 32;   // red holds 2 NW words
     uint32_t mk = 0, mv = 0;
     const int np = (Ls + p.L.P - 1) / p.L.P;
     // warp w takes 32 pages at a time (pages w*32 + 8*32*k + q), their ids loaded
@@ -311,12 +326,12 @@ __device__ void sequence_scale_exps(const PrefillParams& p, int b, int hh, int L
     __syncthreads();   // `red` may still be read by the previous block's epilogue
     if (lane == 0) {
         red[warp] = mk;
-        red[8 + warp] = mv;
+        red[NW + warp] = mv;
     }
     __syncthreads();
-    for (int w = 0; w < kPrefillThreads / 32; w++) {
+    for (int w = 0; w < NW; w++) {
         mk = max(mk, red[w]);
-        mv = max(mv, red[8 + w]);
+        mv = max(mv, red[NW + w]);
     }
     *ek = scale_exp_of_bits<KK>(mk);
     *ev = scale_exp_of_bits<KV>(mv);
@@ -326,11 +341,11 @@ __device__ void sequence_scale_exps(const PrefillParams& p, int b, int hh, int L
 // (sequence, kv-head), i.e. query token (R0 + r) / G, head (R0 + r) % G.  fp16
 // (rotated by the Hadamard-256 first when K is rotated), or the bf16 bits
 // themselves for BF16 keys; rows past the chunk are zeros.  One warp per row.
-template <int D, bool QBF16>
+template <int D, bool QBF16, int NT = kPrefillThreads>
 __device__ __forceinline__ void stage_q(const PrefillParams& p, uint8_t* sQ, float* qrm, int64_t qrow0, int hh,
                                         int64_t R0, int64_t rows_total, int warp, int lane) {
     constexpr int EPL = D / 32;
-    for (int r = warp; r < kPrefillRows; r += kPrefillThreads / 32) {
+    for (int r = warp; r < kPrefillRows; r += NT / 32) {
         const int64_t gr = R0 + r;
         uint32_t bits[EPL / 2];
 #pragma unroll
@@ -691,6 +706,425 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(const Prefi
     if (warp == 0) tc::dealloc(tmem, kCols);
 }
 
+
+// ------------------------------------------------------------ warp-specialised kernel
+//
+// Same computation, same tiles, same arithmetic per value, with the work split
+// by role so that the tensor core, the softmax and the dequantisation overlap:
+//  * warp 0 (one thread) issues the products.  Tile order S(0), S(1), PV(0),
+//    S(2), PV(1), ...: S(k + 1) runs while the softmax of tile k does.
+//  * warps 4..7 run the softmax, one query row per thread (its tensor-memory
+//    lane): a thread loads its whole row of S, so no row maximum is exchanged.
+//    O in tensor memory is rescaled (lazily, as above) by its row's thread,
+//    after the previous P V is done and before the next is issued.
+//  * warps 1..3 and 8..15 dequantise key and value tiles straight from the page slabs
+//    in global memory (the next tile's codes are loaded while this tile's are
+//    converted) into double-buffered fp16 operand tiles.
+//  * all warps stage q and store the output between query blocks.
+// Key, value, S and P buffers are double-buffered; the hand-offs go through
+// mbarriers -- kfull/vfull (dequant -> MMA, 11 arrivals), kfree/sfull/pvdone
+// (tcgen05.commit), sfree/pfull (softmax -> MMA, 4 arrivals) -- whose phase
+// parities follow the CTA's running tile count g: buffer g & 1, phase
+// (g >> 1) & 1.  Every wait is bounded; a wait that gives up sets the abort
+// flag, after which every role leaves its loop.
+
+constexpr int kWsThreads = 512;
+constexpr int kDqWarps = 11;      // dequantising warps: 1..3 and 8..15
+constexpr int kWsBars = 15;       // kfull[2] vfull[2] kfree[2] sfull[2] sfree[2] pfull[2] pvdone[2] drain
+
+// A dequantising thread's share of one key or value tile, read from the page
+// slab in global memory.  The tile's T x CPR 16-byte chunks are taken in
+// blocks of 8 rows x 4 chunks, one block per warp and step: lane l holds row
+// 8 rb + l % 8, chunk 4 cb + l / 8.  So a warp's loads cover 64 contiguous
+// bytes of each of 8 rows, and each 8-lane phase of its 16-byte shared-memory
+// stores writes one chunk column of 8 consecutive rows -- consecutive 16-byte
+// slots of the operand tile, free of bank conflicts.  Rows at or past `valid`
+// load as zero codes with zero scales, which dequantise to zeros.
+template <int KIND, int D>
+struct DqShare {
+    static constexpr int CB = row_code_bytes(KIND, D), SB = row_scale_bytes(KIND, D);
+    static constexpr int CPR = CB / 16;                // chunks per row: 4 .. 32
+    static constexpr int NW = kDqWarps;
+    static constexpr int NPT = ((kMaxT / 8) * (CPR / 4) + NW - 1) / NW;   // blocks per warp at T = 64
+    uint4 w[NPT > 0 ? NPT : 1];
+    uint32_t sb[NPT > 0 ? NPT : 1];
+
+    // lgR = log2(T / 8): the tile's row blocks
+    __device__ __forceinline__ static void chunk_of(int i, int lgR, int dw, int l, int& t, int& j, bool& in) {
+        const int id = dw + i * NW;                    // block id
+        in = id < ((CPR / 4) << lgR);
+        t = ((id & ((1 << lgR) - 1)) << 3) + (l & 7);
+        j = ((id >> lgR) << 2) + (l >> 3);
+    }
+    __device__ __forceinline__ void fetch(const uint8_t* codes, const uint8_t* scales, int r0, int lgR, int valid,
+                                          int dw, int l) {
+#pragma unroll
+        for (int i = 0; i < NPT; i++) {
+            int t, j;
+            bool in;
+            chunk_of(i, lgR, dw, l, t, j, in);
+            w[i] = make_uint4(0, 0, 0, 0);
+            sb[i] = 0;
+            if (in && t < valid) {
+                const int row = r0 + t;
+                w[i] = __ldg(reinterpret_cast<const uint4*>(codes + (int64_t)row * CB +
+                                                            ((j ^ row_swizzle(KIND, D, row)) << 4)));
+                if constexpr (SB > 0) {
+                    const uint8_t* srow = scales + (int64_t)row * SB;
+                    if constexpr (kind_scale_bytes(KIND) == 2 || kind_bits(KIND) == 4) {
+                        const int off = kind_bits(KIND) == 4 ? 2 * j : 2 * (j * 16 / kind_group(KIND));
+                        sb[i] = __ldg(reinterpret_cast<const uint16_t*>(srow + off));
+                    } else {
+                        sb[i] = __ldg(srow + j * 16 / kind_group(KIND));
+                    }
+                }
+            }
+        }
+    }
+    __device__ __forceinline__ void store(uint8_t* tile, int T, int lgR, int dw, int l, float smul) const {
+#pragma unroll
+        for (int i = 0; i < NPT; i++) {
+            int t, j;
+            bool in;
+            chunk_of(i, lgR, dw, l, t, j, in);
+            if (in) dequant_chunk<KIND, D>(w[i], sb[i], j, tile, t, T, smul);
+        }
+    }
+};
+
+template <int KK, int KV, int D>
+__global__ void __launch_bounds__(kWsThreads, 1) prefill_ws_kernel(const PrefillParams p) {
+    constexpr bool KBF = (KK == RK_BF16RAW);
+    constexpr int EPL = D / 32;
+    constexpr int OST = D + 4;
+    constexpr uint32_t kCols = D == 256 ? 512 : 256;   // O in [0, D), S(b) in [D + 64 b, D + 64 b + 64)
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const int T = p.T, lgR = 28 - __clz(T);       // log2(T / 8)
+    uint8_t* sQ = smem;
+    uint8_t* sK0 = sQ + kPrefillRows * D * 2;     // sK(b) = sK0 + b T D 2
+    uint8_t* sV0 = sK0 + 2 * T * D * 2;
+    uint8_t* sP0 = sV0 + 2 * T * D * 2;           // sP(b) = sP0 + b 128 T 2
+    float* sO = reinterpret_cast<float*>(smem);   // epilogue staging, over the operand tiles
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + prefill_ws_region(D, T));
+    float* qrm = reinterpret_cast<float*>(bars + kWsBars + 1);
+    uint32_t* red = reinterpret_cast<uint32_t*>(qrm + kPrefillRows);   // [32]
+    uint32_t* tslot = red + 32;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
+    enum { KFULL = 0, VFULL = 2, KFREE = 4, SFULL = 6, SFREE = 8, PFULL = 10, PVDONE = 12, DRAIN = 14 };
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    int64_t idx = blockIdx.x;
+    const int slot = (int)(idx % p.slots);
+    idx /= p.slots;
+    const int hh = (int)(idx % p.L.H);
+    const int b = (int)(idx / p.L.H);
+    const int64_t qrow0 = p.cu_q_lens[b];
+    const int n = max(0, p.cu_q_lens[b + 1] - (int)qrow0);
+    const int Ls = p.seq_lens[b];
+    const int64_t rows_total = (int64_t)n * p.G;
+    const int64_t nblk = (rows_total + kPrefillRows - 1) / kPrefillRows;
+    if (slot >= nblk) return;
+
+    auto bar = [&](int i) { return smem_addr(&bars[i]); };
+    if (tid == 0) {
+        for (int i = 0; i < kWsBars; i++)
+            mbar_init(bar(i), i < KFREE ? (uint32_t)kDqWarps : (i >= SFREE && i < PVDONE) ? 4u : 1u);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 0) tc::alloc(smem_addr(tslot), kCols);
+    tc::fence_before();
+    __syncthreads();
+    tc::fence_after();
+    const uint32_t tmem = *tslot;
+    const uint32_t tO = tmem;
+    auto tS = [&](uint32_t bb) { return tmem + D + 64 * bb; };
+    auto sK = [&](uint32_t bb) { return sK0 + bb * T * D * 2; };
+    auto sV = [&](uint32_t bb) { return sV0 + bb * T * D * 2; };
+    auto sP = [&](uint32_t bb) { return sP0 + bb * kPrefillRows * T * 2; };
+    // a bounded wait taken by every lane of the warp alike
+    auto wait_warp = [&](int i, uint32_t phase) {
+        bool ok = mbar_wait(bar(i), phase, abort_flag, p.wait_polls);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok && lane == 0) atomicOr(p.status, kStatusWaitTimeout);
+        return ok;
+    };
+
+    auto block_tiles = [&](int64_t jb) {
+        const int64_t R0 = (nblk - 1 - jb) * kPrefillRows;   // the heaviest block first
+        const int64_t r_last = min(R0 + kPrefillRows, rows_total) - 1;
+        const int pos_hi = Ls - n + (int)(r_last / p.G);
+        return pos_hi >= 0 ? pos_hi / T + 1 : 0;
+    };
+
+    int ek_seq = 0, ev_seq = 0;
+    if constexpr (scale_normalised(KK) || scale_normalised(KV))
+        sequence_scale_exps<KK, KV, D, kWsThreads>(p, b, hh, Ls, red, &ek_seq, &ev_seq);
+    const float kmul = pow2i(-ek_seq), vmul = pow2i(-ev_seq);
+
+    // where key tile k of the sequence lives: the block-table entry of its page
+    // (-1 past the table's width), then its page slab and first row there
+    auto tile_pid = [&](int k) -> int {
+        const int page = k * T / p.L.P;
+        return page < p.max_pages ? p.block_table[(int64_t)b * p.max_pages + page] : -1;
+    };
+    auto tile_slab = [&](int pid, int k, int& r0) -> const uint8_t* {
+        const int t0 = k * T;
+        r0 = t0 % p.L.P;
+        if (pid < 0 || pid >= p.L.num_pages) {
+            if ((threadIdx.x & 31) == 0) atomicOr(p.status, kStatusBadPage);
+            pid = 0;
+        }
+        return p.slabs + ((int64_t)pid * p.L.H + hh) * p.L.slab;
+    };
+
+    const uint32_t idS = tc::idesc_f16(KBF, false, T), idO = tc::idesc_f16(false, true, D);
+    uint32_t gk = 0;      // key tiles of earlier query blocks (every role counts alike)
+    float l_row = 0.f;    // softmax threads: the row's sum of weights
+    for (int64_t jb = slot; jb < nblk; jb += p.slots) {
+        const int64_t R0 = (nblk - 1 - jb) * kPrefillRows;
+        const int ntiles = block_tiles(jb);
+        stage_q<D, KBF, kWsThreads>(p, sQ, qrm, qrow0, hh, R0, rows_total, warp, lane);
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncthreads();   // q staged
+
+        if (warp == 0) {
+            // ---- the products, issued by one thread
+            if (lane == 0 && ntiles > 0) {
+                const uint32_t aQ = smem_addr(sQ);
+                auto wait1 = [&](int i, uint32_t phase) {
+                    const bool ok = mbar_wait(bar(i), phase, abort_flag, p.wait_polls);
+                    if (!ok) atomicOr(p.status, kStatusWaitTimeout);
+                    return ok;
+                };
+                for (int k = 0; k <= ntiles; k++) {
+                    if (k < ntiles) {
+                        const uint32_t g = gk + k, bb = g & 1u, ph = (g >> 1) & 1u;
+                        if (!wait1(KFULL + bb, ph)) break;
+                        if (k >= 2 && !wait1(SFREE + bb, ph ^ 1u)) break;   // softmax of tile g - 2 done
+                        tc::fence_after();
+                        const uint32_t aK = smem_addr(sK(bb));
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; kk++)
+                            tc::mma_f16(tS(bb), tc::sdesc(aQ + 256 * kk, 128, 16 * D),
+                                        tc::sdesc(aK + kk * 32 * T, 16 * T, 128), idS, kk > 0);
+                        tc::commit(bar(SFULL + bb));
+                        tc::commit(bar(KFREE + bb));
+                    }
+                    if (k >= 1) {
+                        const uint32_t g = gk + k - 1, bb = g & 1u, ph = (g >> 1) & 1u;
+                        if (!wait1(PFULL + bb, ph) || !wait1(VFULL + bb, ph)) break;
+                        tc::fence_after();
+                        const uint32_t aP = smem_addr(sP(bb)), aV = smem_addr(sV(bb));
+#pragma unroll
+                        for (int kk = 0; kk < kMaxT / 16; kk++)
+                            if (kk < T / 16)
+                                tc::mma_f16(tO, tc::sdesc(aP + kk * 2 * (kPrefillRows * 16), kPrefillRows * 16, 128),
+                                            tc::sdesc(aV + 256 * kk, 128, 16 * T), idO, k > 1 || kk > 0);
+                        tc::commit(bar(PVDONE + bb));
+                    }
+                }
+            }
+        } else if (warp >= 4 && warp < 8) {
+            // ---- softmax: thread = row r, tensor-memory lane r
+            const int g4 = warp & 3, r = g4 * 32 + lane;
+            const uint32_t lane_bits = (uint32_t)(g4 * 32) << 16;
+            const int64_t gr = R0 + r;
+            const int pos = gr < rows_total ? Ls - n + (int)(gr / p.G) : -1;
+            const int64_t gfirst = R0 + g4 * 32;
+            const int gpos_min = gfirst + 31 < rows_total ? Ls - n + (int)(gfirst / p.G) : -1;
+            const float qm = p.q_mult * pow2i(ek_seq) * qrm[r];
+            float m_ref = -INFINITY;
+            l_row = 0.f;
+            bool ok = true;
+            for (int k = 0; k < ntiles && ok; k++) {
+                const uint32_t g = gk + k, bb = g & 1u, ph = (g >> 1) & 1u;
+                if (!(ok = wait_warp(SFULL + bb, ph))) break;
+                tc::fence_after();
+                uint32_t v[64];
+                tc::ld32(tS(bb) + lane_bits, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+                if (T > 32) {
+                    tc::ld32(tS(bb) + lane_bits + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+                } else {
+#pragma unroll
+                    for (int i = 32; i < 64; i++) v[i] = 0u;
+                }
+                tc::wait_ld();
+                tc::fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(SFREE + bb));   // S(b) may be overwritten
+                const int t0 = k * T;
+                const bool mask = t0 + T - 1 > gpos_min;
+                float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // four chains for latency
+#pragma unroll
+                for (int i = 0; i < 64; i++) {
+                    float x = __uint_as_float(v[i]) * qm;
+                    if (i >= T || (mask && t0 + i > pos)) x = -INFINITY;
+                    v[i] = __float_as_uint(x);
+                    mx4[i & 3] = fmaxf(mx4[i & 3], x);
+                }
+                const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+                float corr = 1.f;
+                const bool resc = mx > m_ref + 8.f;
+                if (resc) {
+                    corr = ex2(m_ref - mx);
+                    m_ref = mx;
+                }
+                const float base = m_ref == -INFINITY ? 0.f : m_ref;
+                float rs4[4] = {0.f, 0.f, 0.f, 0.f};
+                uint8_t* pt = sP(bb);
+#pragma unroll
+                for (int q8 = 0; q8 < 8; q8++) {
+                    uint32_t hw[4];
+#pragma unroll
+                    for (int i = 0; i < 4; i++) {
+                        const float pa = ex2(__uint_as_float(v[8 * q8 + 2 * i]) - base);
+                        const float pb = ex2(__uint_as_float(v[8 * q8 + 2 * i + 1]) - base);
+                        rs4[i] += pa + pb;
+                        hw[i] = f16x2_of(pa, pb);
+                    }
+                    if (8 * q8 < T) *reinterpret_cast<uint4*>(pt + p_off(r, 8 * q8)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                }
+                l_row = l_row * corr + ((rs4[0] + rs4[1]) + (rs4[2] + rs4[3]));
+                if (k > 0 && __any_sync(0xffffffffu, resc)) {
+                    // O of this row times corr, once the previous P V has landed in it
+                    const uint32_t gp = g - 1;
+                    if (!(ok = wait_warp(PVDONE + (gp & 1u), (gp >> 1) & 1u))) break;
+                    tc::fence_after();
+#pragma unroll 1
+                    for (int cc = 0; cc < D; cc += 32) {
+                        uint32_t o[32];
+                        tc::ld32(tO + lane_bits + cc, o);
+                        tc::wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; i++) o[i] = __float_as_uint(__uint_as_float(o[i]) * corr);
+                        tc::st32(tO + lane_bits + cc, o);
+                    }
+                    tc::wait_st();
+                }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                tc::fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(PFULL + bb));
+            }
+            if (ok && ntiles > 0) {   // the block's last P V
+                const uint32_t gl = gk + ntiles - 1;
+                if (wait_warp(PVDONE + (gl & 1u), (gl >> 1) & 1u)) tc::fence_after();
+            }
+        } else {
+            // ---- dequantisation of key and value tiles, straight from the slabs
+            const int dw = warp < 4 ? warp - 1 : warp - 5;   // dequantising warp 0..10
+            DqShare<KK, D> rk;
+            DqShare<KV, D> rv;
+            // tile k + 1's codes are loaded while tile k is converted, and tile
+            // k + 2's block-table entry with them, so no load waits on another
+            int r0 = 0;
+            const uint8_t* slab = ntiles > 0 ? tile_slab(tile_pid(0), 0, r0) : p.slabs;
+            int pid_next = ntiles > 1 ? tile_pid(1) : 0;
+            int valid = min(T, Ls);
+            if (ntiles > 0) {
+                rk.fetch(slab, slab + p.L.off_ks, r0, lgR, valid, dw, lane);
+                rv.fetch(slab + p.L.off_vc, slab + p.L.off_vs, r0, lgR, valid, dw, lane);
+            }
+            for (int k = 0; k < ntiles; k++) {
+                const uint32_t g = gk + k, bb = g & 1u, ph = (g >> 1) & 1u;
+                if (k >= 2 && !wait_warp(KFREE + bb, ph ^ 1u)) break;   // S of tile g - 2 done with sK(b)
+                rk.store(sK(bb), T, lgR, dw, lane, kmul);
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(KFULL + bb));
+                int r1 = 0;
+                const uint8_t* slab1 = slab;
+                if (k + 1 < ntiles) {
+                    slab1 = tile_slab(pid_next, k + 1, r1);
+                    valid = min(T, Ls - (k + 1) * T);
+                    rk.fetch(slab1, slab1 + p.L.off_ks, r1, lgR, valid, dw, lane);
+                    pid_next = k + 2 < ntiles ? tile_pid(k + 2) : 0;
+                }
+                if (k >= 2 && !wait_warp(PVDONE + bb, ph ^ 1u)) break;   // P V of tile g - 2 done with sV(b)
+                rv.store(sV(bb), T, lgR, dw, lane, vmul);
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(VFULL + bb));
+                if (k + 1 < ntiles) rv.fetch(slab1 + p.L.off_vc, slab1 + p.L.off_vs, r1, lgR, valid, dw, lane);
+            }
+        }
+        gk += (uint32_t)ntiles;
+
+        // ---- epilogue: normalise, stage the rows, rotate V back, store
+        tc::fence_before();
+        __syncthreads();   // every product of the block done; the operand tiles are free
+        tc::fence_after();
+        if (warp >= 4 && warp < 8) {
+            const int g4 = warp & 3, r = g4 * 32 + lane;
+            const uint32_t lane_bits = (uint32_t)(g4 * 32) << 16;
+            const float inv = l_row > 0.f ? p.o_mult / l_row * pow2i(ev_seq) : 0.f;   // O is in units of 2^ev_seq
+            float* so = sO + r * OST;
+            const bool have = __all_sync(0xffffffffu, ntiles > 0 && !*abort_flag);
+#pragma unroll 1
+            for (int cc = 0; cc < D; cc += 32) {
+                uint32_t v[32];
+                if (have) {
+                    tc::ld32(tO + lane_bits + cc, v);
+                    tc::wait_ld();
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; i++) v[i] = 0u;
+                }
+#pragma unroll
+                for (int i = 0; i < 32; i += 4)
+                    *reinterpret_cast<float4*>(so + cc + i) =
+                        make_float4(__uint_as_float(v[i]) * inv, __uint_as_float(v[i + 1]) * inv,
+                                    __uint_as_float(v[i + 2]) * inv, __uint_as_float(v[i + 3]) * inv);
+            }
+        }
+        tc::fence_before();
+        __syncthreads();   // output rows staged; tensor memory reads done
+        for (int rr = warp; rr < kPrefillRows; rr += kWsThreads / 32) {
+            const int64_t grr = R0 + rr;
+            if (grr >= rows_total) break;
+            float x[EPL];
+#pragma unroll
+            for (int i = 0; i < EPL; i += 4) {
+                const float4 v = *reinterpret_cast<const float4*>(sO + rr * OST + lane * EPL + i);
+                x[i] = v.x; x[i + 1] = v.y; x[i + 2] = v.z; x[i + 3] = v.w;
+            }
+            if constexpr (D == 256) {
+                if (p.rot_v) fwht256_warp(x, lane);
+            }
+            const int64_t i_tok = grr / p.G, gq = grr % p.G;
+            const int64_t o = ((qrow0 + i_tok) * p.Hq + (int64_t)hh * p.G + gq) * D + lane * EPL;
+            if (p.out_fp32) {
+                float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + o);
+#pragma unroll
+                for (int i = 0; i < EPL / 4; i++) dst[i] = make_float4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
+            } else {
+                uint32_t hb[EPL / 2];
+#pragma unroll
+                for (int i = 0; i < EPL / 2; i++) hb[i] = bf16x2_of(x[2 * i], x[2 * i + 1]);
+                uint16_t* dst = static_cast<uint16_t*>(p.out) + o;
+                if constexpr (EPL == 8) {
+                    *reinterpret_cast<uint4*>(dst) = make_uint4(hb[0], hb[1], hb[2], hb[3]);
+                } else {
+                    *reinterpret_cast<uint2*>(dst) = make_uint2(hb[0], hb[1]);
+                }
+            }
+        }
+        __syncthreads();   // the shared region is free for the next block
+    }
+    // every product issued has completed before the tensor memory is freed
+    // (on a normal exit they have; after a wait gave up, wait -- bounded -- here)
+    if (tid == 0) {
+        tc::commit(bar(DRAIN));
+        int ignore = 0;
+        (void)mbar_wait(bar(DRAIN), 0, &ignore);
+    }
+    tc::fence_before();
+    __syncthreads();
+    tc::fence_after();
+    if (warp == 0) tc::dealloc(tmem, kCols);
+}
+
 }  // namespace
 
 // ------------------------------------------------------------ host side
@@ -705,10 +1139,24 @@ static constexpr size_t kSmemLimit = 227 * 1024;   // opt-in shared memory per C
 cudaError_t plan_prefill(const Layout& L, PrefillPlan* plan) {
     int T = 64;
     while (L.P % T) T >>= 1;   // the largest of 64, 32, 16 that divides the page
+    {
+        // the warp-specialised kernel, whenever its tiles fit
+        PrefillPlan q;
+        memset(&q, 0, sizeof(q));
+        q.T = T;
+        q.kernel = 1;
+        q.smem = (size_t)prefill_ws_smem(L.D, T);
+        if (q.smem <= kSmemLimit) {
+            *plan = q;
+            return cudaSuccess;
+        }
+    }
     const int stages = 2;
     for (;;) {
         PrefillPlan q;
+        memset(&q, 0, sizeof(q));
         q.T = T;
+        q.kernel = 0;
         q.stages = stages;
         q.st_ks = (int)align16((int64_t)T * L.kc);
         q.st_vc = q.st_ks + (int)align16((int64_t)T * L.ks);
@@ -726,10 +1174,11 @@ cudaError_t plan_prefill(const Layout& L, PrefillPlan* plan) {
 
 template <int KK, int KV, int D>
 static cudaError_t launch_t(const PrefillParams& p, const PrefillPlan& plan, int64_t grid, cudaStream_t s) {
-    auto kern = prefill_kernel<KK, KV, D>;
+    auto kern = plan.kernel == 1 ? prefill_ws_kernel<KK, KV, D> : prefill_kernel<KK, KV, D>;
+    const int threads = plan.kernel == 1 ? kWsThreads : kPrefillThreads;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan.smem);
     if (e != cudaSuccess) return e;
-    kern<<<(unsigned)grid, kPrefillThreads, plan.smem, s>>>(p);
+    kern<<<(unsigned)grid, threads, plan.smem, s>>>(p);
     return cudaGetLastError();
 }
 

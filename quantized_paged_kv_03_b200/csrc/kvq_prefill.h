@@ -23,6 +23,18 @@ KVQ_HD constexpr int64_t prefill_region0(int D, int T) {
 // (128 floats), the tensor-memory address and the abort flag.
 KVQ_HD constexpr int64_t prefill_tail_bytes(int stages) { return 8 * (stages + 2) + 3 * kPrefillRows * 4 + 16; }
 
+// The warp-specialised kernel's shared memory: q (128 x D), double-buffered
+// key and value tiles (T x D each) and P (128 x T), all 16-bit -- or, if larger,
+// the fp32 output rows (128 x (D + 4)) of the epilogue -- rounded up to 1 KB;
+// then 16 mbarriers, the rows' q multipliers (128 floats), a 32-word exchange
+// buffer, the tensor-memory address and the abort flag.
+KVQ_HD constexpr int64_t prefill_ws_region(int D, int T) {
+    const int64_t ops = ((int64_t)kPrefillRows * D + 4 * (int64_t)T * D + 2 * (int64_t)kPrefillRows * T) * 2;
+    const int64_t osm = (int64_t)kPrefillRows * (D + 4) * 4;
+    return ((ops > osm ? ops : osm) + 1023) & ~int64_t(1023);
+}
+KVQ_HD constexpr int64_t prefill_ws_smem(int D, int T) { return prefill_ws_region(D, T) + 16 * 8 + kPrefillRows * 4 + 32 * 4 + 16; }
+
 struct PrefillParams {
     Layout L;
     const uint8_t* slabs;        // first slab of the layer
@@ -47,6 +59,7 @@ struct PrefillParams {
 };
 
 struct PrefillPlan {
+    int kernel;                  // 1: warp-specialised (prefill_ws_kernel), 0: every warp in every phase
     int T, stages;
     int st_ks, st_vc, st_vs, st_bytes;
     size_t smem;
