@@ -53,14 +53,14 @@ def make_l2_flush(torch):
 # From an ncu capture of the fused step's decode_kernel launch on the headline
 # workload: DRAM bytes read + written per launch.  It describes the kernel built
 # from the sources with this digest only (null for any other build).
-HEADLINE_TRAFFIC = {"bytes": 125_782_016 + 3_462_400,
-                    "sources_sha256": "4f98db180293a36848fe190003cdd9c8250b5f04952ab6c1524610d9eaa02f2f"}
+HEADLINE_TRAFFIC = {"bytes": 127_485_850 + 3_760_623,
+                    "sources_sha256": "61de776ca4d12f8e4791609c36e120eda98c3ebd84ab62ea4053c263cb646104"}
 KERNEL_SOURCES = ("kvq_decode.cu", "kvq_common.cuh", "kvq_quant.cuh", "kvq_internal.h")
 
 
 # The same for the chunked-prefill kernel on its workload.
-PREFILL_TRAFFIC = {"bytes": 175_584_768 + 42_600_960,
-                   "sources_sha256": "8018ed37346010a003d7008da643f155893e94e2f5dc68613458ca8b46a53099"}
+PREFILL_TRAFFIC = {"bytes": 174_266_304 + 38_802_581,
+                   "sources_sha256": "46b0347d5dd9dbdca03eadd045e896d025ed3e6212f789adc117604d5f9eefb4"}
 PREFILL_SOURCES = ("kvq_prefill.cu", "kvq_prefill.h", "kvq_tc.cuh", "kvq_common.cuh")
 
 
@@ -393,7 +393,7 @@ class PrefillArm:
             "flops_per_launch": self.flops,
             "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": peak_tflops,
                          "unit": "TFLOP/s", "frac": round(tflops / peak_tflops, 4), "traffic": prefill_traffic(),
-                         "kernel": "prefill_kernel (tcgen05)", "peak_source": f"{peak_kind} bf16_tflops"},
+                         "kernel": "prefill_ws_kernel (tcgen05, warp-specialised)", "peak_source": f"{peak_kind} bf16_tflops"},
             "gpu_launches_per_step": 2,
         }
 
