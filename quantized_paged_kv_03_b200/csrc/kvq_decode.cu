@@ -310,27 +310,23 @@ __device__ __forceinline__ void store_out(void* out, int out_fp32, int64_t ob, c
     }
 }
 
-// Grid-wide barrier of the G co-resident CTAs (cooperative launch).  Arrival
-// counter + generation word in the workspace; the last arriver resets the
-// counter, so it is zero again after every launch.  Every CTA arrives; only a
-// CTA that passes `wait` waits for the others.  The wait is bounded: on
-// timeout the CTA records it and returns false.
+// One-use grid barrier of a launch over G CTAs: bar[0] counts arrivals,
+// bar[2] departures; both are zero between launches (the last CTA to leave
+// resets them), so a waiter needs no generation word: it polls until all G
+// have arrived.  A CTA that needs nothing from the others (`wait` false) only
+// counts itself in and out.  Bounded: a waiter gives up after 2^26 polls and
+// returns false (the caller records the timeout).
 __device__ __forceinline__ bool grid_barrier(unsigned* bar, unsigned G, int* flag_smem, bool wait) {
     __syncthreads();
     if (threadIdx.x == 0) {
-        volatile unsigned* vgen = bar + 1;
-        const unsigned gen = *vgen;
-        __threadfence();
+        __threadfence();   // this CTA's partials before its arrival
         const unsigned old = atomicAdd(bar, 1u);
         int ok = 1;
-        if (old == G - 1) {
-            atomicExch(bar, 0u);
-            __threadfence();
-            atomicAdd(bar + 1, 1u);
-        } else if (wait) {
+        if (wait && old != G - 1) {
+            volatile unsigned* arrivals = bar;
             long it = 0;
-            while (*vgen == gen) {
-                __nanosleep(64);
+            while (*arrivals < G) {
+                __nanosleep(32);
                 if (++it > (1l << 26)) {
                     ok = 0;
                     break;
@@ -338,6 +334,11 @@ __device__ __forceinline__ bool grid_barrier(unsigned* bar, unsigned G, int* fla
             }
         }
         __threadfence();
+        // every CTA has left the wait once departures reach G: reset for the next launch
+        if (atomicAdd(bar + 2, 1u) == G - 1) {
+            atomicExch(bar, 0u);
+            atomicExch(bar + 2, 0u);
+        }
         *flag_smem = ok;
     }
     __syncthreads();
@@ -1317,7 +1318,7 @@ static size_t partial_bytes(const Layout& L, int grid) {
     return (((size_t)grid * 2 * (16 + 8 * (size_t)L.D) * sizeof(float)) + 255) & ~(size_t)255;
 }
 
-// Zeroed region: the grid barrier's two words, then one counter per CTA (the
+// Zeroed region: the grid barrier's words (256 bytes), then one counter per CTA (the
 // parts of the cut segment that ends in that CTA's range).
 static size_t zero_bytes(int grid) { return (256 + 4 * (size_t)grid + 255) & ~(size_t)255; }
 

@@ -73,7 +73,7 @@ struct DecodeParams {
     bool rot_k, rot_v;
     long wait_polls;             // polls of a pipeline wait before it gives up
     float* partials;             // [gridDim.x][2][16 + 8 * D]: (max, sum, output) of cut segments
-    unsigned* barrier;           // grid barrier: [0] arrivals (zero between calls), [1] generation
+    unsigned* barrier;           // grid barrier: [0] arrivals, [2] departures (zero between calls)
     unsigned* seg_count;         // [gridDim.x] parts counted in of the cut segment ending in each CTA's range
     uint32_t* status;
     int stages;                  // pipeline depth (page slabs in shared memory)
