@@ -231,7 +231,9 @@ int kvq::decode_setup(kvq_cache* cache, int32_t layer, const void* k_new, const 
     p.rot_v = rot_of(cache, 1);
     p.wait_polls = kvq::wait_polls();
     p.partials = nullptr;
-    p.barrier = nullptr;
+    p.group_partials = nullptr;
+    p.grp_count = nullptr;
+    p.seg_groups = nullptr;
     p.status = (uint32_t*)cache->pool;
     p.k_new = (const uint16_t*)k_new;
     p.v_new = (const uint16_t*)v_new;
@@ -254,8 +256,9 @@ int kvq::decode_launch(DecodeParams* p, const DecodePlan& plan, void* workspace,
     size_t zoff = 0, zbytes = 0;
     decode_workspace_zero_region(p->L, p->B, p->HB, plan.grid, &zoff, &zbytes);
     p->partials = (float*)workspace;
-    p->barrier = (unsigned*)((uint8_t*)workspace + zoff);
-    p->seg_count = p->barrier + 64;   // after the barrier's 256-byte block
+    p->group_partials = p->partials + (size_t)plan.grid * 2 * (16 + 8 * (size_t)p->L.D);
+    p->grp_count = (unsigned*)((uint8_t*)workspace + zoff);
+    p->seg_groups = p->grp_count + plan.grid;
     return cuda_status(launch_decode(*p, plan, stream));
 }
 

@@ -8,31 +8,30 @@
 // not arithmetic) make this a streaming kernel: its roofline is HBM bandwidth.
 //
 // Design (B200, sm_100a):
-//  * Persistent cooperative grid, 8 warps per CTA (three CTAs per SM where a
-//    64-token unit is small enough, else two).  The work units of the whole
+//  * Persistent grid of two 8-warp CTAs per SM.  The work units of the whole
 //    batch -- a page of one kv-head, or a 64-token span of a larger page --
 //    ordered (sequence, kv-head, 8-head block, unit), are cut into gridDim.x
 //    contiguous ranges of equal cost, where a unit costs 1 and every segment a
-//    range touches adds the fixed price of its start and end; ragged batches
-//    balance to within about one unit.
+//    range touches adds the fixed price of its start, end and merge; ragged
+//    batches balance to within about one unit.
 //  * A whole-page unit (K codes, K scales, V codes, V scales of one kv-head:
 //    one contiguous range in HBM) arrives with ONE cp.async.bulk into a
 //    shared-memory stage; a span of a larger page with one copy per part.
 //    Completion is tracked by an mbarrier.  Warps release a stage with a
 //    shared counter; the last warp to release it issues the next copy into it,
 //    so warps never wait for each other unit by unit.
-//  * A 16-token tile is owned by a warp pair: each warp takes one half of
-//    head_dim.  Codes become fp16 (exact for every format) in registers straight
-//    from shared memory and feed mma.sync m16n8k16 with the GQA group (<= 8
-//    query heads) as N: S^T = K q^T (tokens as M, the pair adds its two halves
-//    through shared memory), then O^T += V^T P^T (head_dim as M; movmatrix
+//  * A warp owns a 16-token tile over all of head_dim.  Codes become fp16
+//    (exact for every format) in registers straight from shared memory and
+//    feed mma.sync m16n8k16 with the GQA group (<= 8 query heads) as N:
+//    S^T = K q^T (tokens as M), then O^T += V^T P^T (head_dim as M; movmatrix
 //    transposes the V and P fragments).  Group scales are folded into fp32
-//    scores (K) or into P (V); NVFP4 scales go into the operand, where
-//    code x scale is exact in fp16.
+//    scores (K) or into P (V, against a power-of-two reference); NVFP4 scales
+//    go into the operand, where code x scale is exact in fp16.
 //  * Online softmax in the log2 domain; the warps merge in shared memory at
 //    the end of each (sequence, kv-head) segment.  A segment cut by a range
-//    boundary leaves a partial (max, sum, unnormalised output); after one grid
-//    barrier every CTA that holds a part merges a share of that segment.
+//    boundary leaves a partial (max, sum, unnormalised output), merged by
+//    whichever CTA counts in last (in groups of kFewParts parts, then the
+//    groups), so no CTA ever waits on another.
 //  * Rotated K: q is rotated by the same normalised Hadamard-256 (orthonormal,
 //    so q.k is unchanged).  Rotated V: the output is rotated back (the matrix
 //    is symmetric and its own inverse).
@@ -42,15 +41,15 @@
 
 namespace kvq {
 
-constexpr int kDecThreads = 256;   // 8 warps: 4 tile slots x 2 head_dim halves
+constexpr int kDecThreads = 256;   // 8 warps, each a 16-token tile over all of head_dim
 // Row stride (floats) of the output-combine buffer: 4 floats of padding per head
 // row spread the heads a warp writes over different banks.
 template <int D>
 constexpr int kOsmStride = D + 4;
 constexpr int kMaxStages = 8;
 constexpr int kMaxBatch = 4096;
-// A cut segment with at most this many parts is merged by the CTA that
-// completes it; one with more is merged by all of its CTAs after a grid barrier.
+// Parts of a cut segment merged together by the CTA that completes them: a
+// segment of more parts is merged in groups of this many, then the groups.
 constexpr int kFewParts = 16;
 constexpr long kWaitPolls = 1l << 22;
 
@@ -310,73 +309,37 @@ __device__ __forceinline__ void store_out(void* out, int out_fp32, int64_t ob, c
     }
 }
 
-// One-use grid barrier of a launch over G CTAs: bar[0] counts arrivals,
-// bar[2] departures; both are zero between launches (the last CTA to leave
-// resets them), so a waiter needs no generation word: it polls until all G
-// have arrived.  A CTA that needs nothing from the others (`wait` false) only
-// counts itself in and out.  Bounded: a waiter gives up after 2^26 polls and
-// returns false (the caller records the timeout).
-__device__ __forceinline__ bool grid_barrier(unsigned* bar, unsigned G, int* flag_smem, bool wait) {
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        __threadfence();   // this CTA's partials before its arrival
-        const unsigned old = atomicAdd(bar, 1u);
-        int ok = 1;
-        if (wait && old != G - 1) {
-            volatile unsigned* arrivals = bar;
-            long it = 0;
-            while (*arrivals < G) {
-                __nanosleep(32);
-                if (++it > (1l << 26)) {
-                    ok = 0;
-                    break;
-                }
-            }
-        }
-        __threadfence();
-        // every CTA has left the wait once departures reach G: reset for the next launch
-        if (atomicAdd(bar + 2, 1u) == G - 1) {
-            atomicExch(bar, 0u);
-            atomicExch(bar + 2, 0u);
-        }
-        *flag_smem = ok;
-    }
-    __syncthreads();
-    return *flag_smem != 0;
-}
 
-// Merge share j of nshares of the partials of one cut segment (CTAs
-// i_first..i_last each left (max, sum, unnormalised output) for up to 8 query
-// heads): this CTA produces float4 outputs [o0, o1) of the segment's gv x D/4.  One pass: each
-// output's threads fold the parts in with a running (max, sum, output) -- the
-// log-sum-exp merge -- then combine their folds by shuffles; no block barrier.
+// Merge P parts of one cut segment -- part k's (max[8], sum[8], unnormalised
+// output [8][D]) at part_ptr(k) -- in the order k = 0, 1, ... (so the result
+// does not depend on which CTA merges, or when).  One pass: each output float4
+// (head g, d4) is folded by tpo threads, each taking every tpo-th part with a
+// running (max, sum, output) -- the log-sum-exp merge, loads of kMergeBatch
+// parts in flight together -- and the threads' folds are combined by
+// shuffles.  The result goes to the output rows (normalised), or, when `dst`
+// is given, to dst as one more part (unnormalised, with its max and sum).
 constexpr int kMergeBatch = 8;   // parts whose loads are in flight together
 
+// Part k lies at first (k = 0), last (k = P - 1), else base + k * stride
+// floats.  Out of line: it runs once or twice per CTA, after the main loop.
 template <int D>
-__device__ __forceinline__ void merge_segment(const float* partials, void* out, int out_fp32, float o_mult, int Hq,
-                                           int Gq, int b, int h, int hb, int64_t seg_w0, int i_first, int i_last,
-                                           Partition part, int j, int nshares) {
+__device__ __noinline__ void merge_parts(const float* first, const float* last, const float* base, int64_t stride,
+                                         int P, float* dst, void* out, int out_fp32, float o_mult, int Hq, int Gq,
+                                         int b, int h, int hb) {
     const int tid = threadIdx.x;
-    const int P = i_last - i_first + 1;
+    auto part_ptr = [&](int k) { return k == 0 ? first : k == P - 1 ? last : base + k * stride; };
     const int gv = min(8, Gq - hb * 8);
-    const int NU = gv * (D / 4);
-    const int o0 = (int)((int64_t)j * NU / nshares), o1 = (int)((int64_t)(j + 1) * NU / nshares);
-    const int no = o1 - o0;
-    if (no <= 0) return;
-    // The segment is the first of every part's range except possibly the first
-    // part's (slot 0 holds a range's first segment, slot 1 its last).
-    const int slot0 = part.start(i_first) >= seg_w0 ? 0 : 1;
-    int tpo = 1;   // threads per output, splitting the parts
+    const int no = gv * (D / 4);   // float4 outputs
+    int tpo = 1;                   // threads per output, splitting the parts
     while (tpo < 32 && tpo * 2 * no <= kDecThreads) tpo *= 2;
     const int per_pass = kDecThreads / tpo;
-    for (int ob = o0; ob < o1; ob += per_pass) {
+    for (int ob = 0; ob < no; ob += per_pass) {
         const int o = ob + tid / tpo, pl = tid % tpo;
-        const bool valid = o < o1;
+        const bool valid = o < no;
         const int g = valid ? o / (D / 4) : 0, d4 = valid ? o % (D / 4) : 0;
         float M = -INFINITY, L = 0.f;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         if (valid) {
-            // parts in groups of kMergeBatch, all loads of a group in flight together
             for (int k0 = pl; k0 < P; k0 += kMergeBatch * tpo) {
                 float mk[kMergeBatch], lk[kMergeBatch];
                 float4 v[kMergeBatch];
@@ -385,7 +348,7 @@ __device__ __forceinline__ void merge_segment(const float* partials, void* out, 
                     const int k = k0 + q * tpo;
                     mk[q] = -INFINITY;
                     if (k < P) {
-                        const float* pk = partials + ((int64_t)(i_first + k) * 2 + (k == 0 ? slot0 : 0)) * (16 + 8 * D);
+                        const float* pk = part_ptr(k);
                         mk[q] = __ldcg(pk + g);
                         lk[q] = __ldcg(pk + 8 + g);
                         v[q] = __ldcg(reinterpret_cast<const float4*>(pk + 16 + g * D) + d4);
@@ -415,10 +378,18 @@ __device__ __forceinline__ void merge_segment(const float* partials, void* out, 
             M = Mn;
         }
         if (valid && pl == 0) {
-            const float inv = (L > 0.f) ? o_mult / L : 0.f;
-            const float x[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
-            const int64_t oo = ((int64_t)b * Hq + h * Gq + hb * 8 + g) * D + 4 * d4;
-            store_out<4>(out, out_fp32, oo, x);
+            if (dst) {
+                *reinterpret_cast<float4*>(dst + 16 + g * D + 4 * d4) = acc;
+                if (d4 == 0) {
+                    dst[g] = M;
+                    dst[8 + g] = L;
+                }
+            } else {
+                const float inv = (L > 0.f) ? o_mult / L : 0.f;
+                const float x[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
+                const int64_t oo = ((int64_t)b * Hq + h * Gq + hb * 8 + g) * D + 4 * d4;
+                store_out<4>(out, out_fp32, oo, x);
+            }
         }
     }
 }
@@ -485,7 +456,7 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
     off += 16 * 4;
     float* qhm = reinterpret_cast<float*>(smem + off);   // [8] score multiplier of each head of the block
     off += 8 * 4;
-    int* flags = reinterpret_cast<int*>(smem + off);     // [0] abort, [2] grid barrier ok
+    int* flags = reinterpret_cast<int*>(smem + off);     // [0] abort, [1] this CTA merges
     off += 16;
     int* pref = reinterpret_cast<int*>(smem + off);      // [B + 1] page prefix
     off += 4 * (size_t)(B + 1);
@@ -1098,7 +1069,7 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
         // ---- a whole segment is normalised and stored here; a segment cut by
         // a range boundary leaves its unnormalised output as this CTA's partial
         // (rotated back already: the Hadamard is linear, so merging commutes
-        // with it) for the merge after the grid barrier.
+        // with it) for the merge after the loop.
         {
             const int64_t seg_w0 = (int64_t)pref[b] * HH + (int64_t)cc.hh * nspans;
             const bool whole = (seg_w0 >= w0) && (seg_w0 + nspans <= w1);
@@ -1154,64 +1125,71 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
         __syncthreads();
     }
 
-    // ---- merge the cut segments.  A segment cut into at most kFewParts parts
-    // is merged by the CTA that completes it -- the last of its parts to count
-    // itself in -- so no CTA waits on another; a segment with more parts is
-    // merged after a grid barrier, a share by every CTA that holds a part.
-    // Every CTA arrives at the barrier; only those with such a share wait.
-    // (A CTA whose cost share holds no unit still arrives: the barrier counts G.)
-    if (G > 1) {
+    // ---- merge the cut segments, with no CTA waiting on another.  A cut
+    // segment's parts (CTAs i_first..i_last) fall in groups of kFewParts
+    // consecutive CTAs; every part counts itself in on its group's counter,
+    // and the last to arrive merges the group.  A segment of one group is
+    // then done; otherwise the group's merge is one more part, counted in on
+    // the segment's counter, and the last group merged merges the groups.
+    // Counters are indexed by the CTA holding the group's (or segment's)
+    // last part -- a CTA ends at most one group of one cut segment -- and
+    // are left zero for the next call.
+    if (G > 1 && n > 0) {
         Cursor c0, c1;
-        if (n > 0) {
-            cursor_locate(c0, w0, pref, B, HH, HB);
-            cursor_locate(c1, w1 - 1, pref, B, HH, HB);
-        }
-        bool wait = false;
-        for (int k = 0; k < (n > 0 ? 2 : 0); k++) {
+        cursor_locate(c0, w0, pref, B, HH, HB);
+        cursor_locate(c1, w1 - 1, pref, B, HH, HB);
+        const int64_t PSZ = 16 + 8 * (int64_t)D;   // floats of one part
+        for (int k = 0; k < 2; k++) {
             const Cursor& c = k == 0 ? c0 : c1;
             if (k == 1 && c1.b == c0.b && c1.hh == c0.hh) break;
             const int64_t seg_w0 = (int64_t)pref[c.b] * HH + (int64_t)c.hh * c.nspans;
             if (seg_w0 >= w0 && seg_w0 + c.nspans <= w1) continue;     // whole: already stored
             const int i_first = part.owner(c.b, c.hh, 0);
             const int i_last = part.owner(c.b, c.hh, c.nspans - 1);
-            if (i_last - i_first + 1 > kFewParts) {
-                wait = true;
-                continue;
-            }
-            // count this part in; the last to arrive merges the segment and
-            // clears its counter for the next call (counters are indexed by the
-            // CTA holding the segment's end, which ends at most one cut segment)
+            const int P = i_last - i_first + 1, Q = (P + kFewParts - 1) / kFewParts;
+            const int g_first = i_first + ((int)blockIdx.x - i_first) / kFewParts * kFewParts;
+            const int g_last = min(i_last, g_first + kFewParts - 1);
             __syncthreads();   // this CTA's partial is written
             if (tid == 0) {
                 __threadfence();
-                const unsigned old = atomicAdd(&p.seg_count[i_last], 1u);
-                flags[1] = (old == (unsigned)(i_last - i_first));
+                const unsigned old = atomicAdd(&p.grp_count[g_last], 1u);
+                flags[1] = (old == (unsigned)(g_last - g_first));
                 if (flags[1]) {
-                    p.seg_count[i_last] = 0u;
+                    p.grp_count[g_last] = 0u;
                     __threadfence();
                 }
             }
             __syncthreads();
-            if (flags[1])
-                merge_segment<D>(p.partials, p.out, p.out_fp32, p.o_mult, p.Hq, p.G, c.b, c.h, c.hb, seg_w0, i_first,
-                                 i_last, part, 0, 1);
-        }
-        if (!grid_barrier(p.barrier, (unsigned)G, &flags[2], wait)) {
-            if (tid == 0) atomicOr(p.status, kStatusWaitTimeout);
-            return;
-        }
-        if (wait) {
-            for (int k = 0; k < 2; k++) {   // (wait is set only when n > 0)
-                const Cursor& c = k == 0 ? c0 : c1;
-                if (k == 1 && c1.b == c0.b && c1.hh == c0.hh) break;
-                const int64_t seg_w0 = (int64_t)pref[c.b] * HH + (int64_t)c.hh * c.nspans;
-                if (seg_w0 >= w0 && seg_w0 + c.nspans <= w1) continue;
-                const int i_first = part.owner(c.b, c.hh, 0);
-                const int i_last = part.owner(c.b, c.hh, c.nspans - 1);
-                if (i_last - i_first + 1 <= kFewParts) continue;
-                merge_segment<D>(p.partials, p.out, p.out_fp32, p.o_mult, p.Hq, p.G, c.b, c.h, c.hb, seg_w0, i_first,
-                                 i_last, part, (int)blockIdx.x - i_first, i_last - i_first + 1);
+            if (!flags[1]) continue;
+            // parts: slot 1 of the segment's first CTA if the segment is its
+            // range's last, else slot 0 (the segment is every other part's first)
+            const int slot0 = part.start(i_first) >= seg_w0 ? 0 : 1;
+            const float* pbase = p.partials + (int64_t)g_first * 2 * PSZ;     // part kk at pbase + 2 kk PSZ
+            const float* pfirst = pbase + (g_first == i_first ? slot0 : 0) * PSZ;
+            const float* plast = p.partials + (int64_t)g_last * 2 * PSZ;
+            if (Q == 1) {
+                merge_parts<D>(pfirst, plast, pbase, 2 * PSZ, P, nullptr, p.out, p.out_fp32, p.o_mult, p.Hq, p.G,
+                               c.b, c.h, c.hb);
+                continue;
             }
+            merge_parts<D>(pfirst, plast, pbase, 2 * PSZ, g_last - g_first + 1, p.group_partials + (int64_t)g_last * PSZ,
+                           p.out, p.out_fp32, p.o_mult, p.Hq, p.G, c.b, c.h, c.hb);
+            __syncthreads();   // the group's merge is written
+            if (tid == 0) {
+                __threadfence();
+                const unsigned old = atomicAdd(&p.seg_groups[i_last], 1u);
+                flags[1] = (old == (unsigned)(Q - 1));
+                if (flags[1]) {
+                    p.seg_groups[i_last] = 0u;
+                    __threadfence();
+                }
+            }
+            __syncthreads();
+            if (!flags[1]) continue;
+            // group qq's merge sits at the CTA of its last part: i_first + 16 qq + 15, the last at i_last
+            const float* gbase = p.group_partials + (int64_t)(i_first + kFewParts - 1) * PSZ;
+            merge_parts<D>(gbase, p.group_partials + (int64_t)i_last * PSZ, gbase, kFewParts * PSZ, Q, nullptr, p.out,
+                           p.out_fp32, p.o_mult, p.Hq, p.G, c.b, c.h, c.hb);
         }
     }
 }
@@ -1314,13 +1292,15 @@ cudaError_t plan_decode(const Layout& L, int B, int HB, int max_seq_len, DecodeP
     return cudaErrorInvalidConfiguration;
 }
 
+// Partials: two per CTA (its range's first and last segment), then one group
+// merge per CTA (the group of parts ending in it), each 16 + 8 D floats.
 static size_t partial_bytes(const Layout& L, int grid) {
-    return (((size_t)grid * 2 * (16 + 8 * (size_t)L.D) * sizeof(float)) + 255) & ~(size_t)255;
+    return (((size_t)grid * 3 * (16 + 8 * (size_t)L.D) * sizeof(float)) + 255) & ~(size_t)255;
 }
 
-// Zeroed region: the grid barrier's words (256 bytes), then one counter per CTA (the
-// parts of the cut segment that ends in that CTA's range).
-static size_t zero_bytes(int grid) { return (256 + 4 * (size_t)grid + 255) & ~(size_t)255; }
+// Zeroed region: two counters per CTA -- the parts counted in of the group
+// ending in it, the groups counted in of the segment ending in it.
+static size_t zero_bytes(int grid) { return (8 * (size_t)grid + 255) & ~(size_t)255; }
 
 size_t decode_workspace_bytes(const Layout& L, int B, int HB, int grid) {
     (void)B;
@@ -1345,8 +1325,9 @@ cudaError_t launch_decode(const DecodeParams& p, const DecodePlan& plan, cudaStr
     // were both slower)
     q.seg_cost = q.U.sp >= 256 ? 2 : 512 / q.U.sp;
     void* args[] = {&q};
-    // cooperative: the merge after the grid barrier needs every CTA resident
-    return cudaLaunchCooperativeKernel(k, dim3(plan.grid), dim3(plan.threads), args, plan.smem, s);
+    // no CTA waits on another (the merges go to whoever finishes last), so a
+    // plain launch: one resident wave by the plan's sizing, not by requirement
+    return cudaLaunchKernel(k, dim3(plan.grid), dim3(plan.threads), args, plan.smem, s);
 }
 
 }  // namespace kvq

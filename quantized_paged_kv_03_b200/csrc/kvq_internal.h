@@ -73,8 +73,9 @@ struct DecodeParams {
     bool rot_k, rot_v;
     long wait_polls;             // polls of a pipeline wait before it gives up
     float* partials;             // [gridDim.x][2][16 + 8 * D]: (max, sum, output) of cut segments
-    unsigned* barrier;           // grid barrier: [0] arrivals, [2] departures (zero between calls)
-    unsigned* seg_count;         // [gridDim.x] parts counted in of the cut segment ending in each CTA's range
+    float* group_partials;       // [gridDim.x][16 + 8 * D]: merge of the group of parts ending in each CTA
+    unsigned* grp_count;         // [gridDim.x] parts counted in of the group ending in each CTA (zero between calls)
+    unsigned* seg_groups;        // [gridDim.x] groups counted in of the segment ending in each CTA (zero between calls)
     uint32_t* status;
     int stages;                  // pipeline depth (page slabs in shared memory)
     int pid_cap;                 // page ids of a CTA's range preloaded into shared memory
