@@ -163,3 +163,20 @@ def test_fused_append_decode_equals_append_then_decode(fmt, cfg, D, P, lengths, 
                              oc.decode(w.q, w.block_table, w.seq_lens, threads=8), w)
     assert ratio <= 1.0, err
     assert fused.read_device_status() == 0
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("fmt,cfg,H,lengths", [("k8v4", 3, 1, [24000]), ("int8_g64", 1, 1, [12000, 9000])],
+                         ids=["one_segment_296_parts", "two_segments"])
+def test_decode_segment_cut_into_many_groups(fmt, cfg, H, lengths):
+    """A single long sequence on one kv-head is cut across every CTA of the
+    grid (hundreds of parts): its parts are merged in groups of 16 and the
+    groups merged again, by whichever CTAs finish last.  The result must match
+    the oracle and be bit-identical on a repeat call (a fixed merge order,
+    counters left at zero)."""
+    w, c, got, want = run_case(fmt, cfg, 256, 64, lengths, H, 6)
+    ratio, err = attn_errors(got, want, w)
+    assert ratio <= 1.0, f"{fmt}: max err {err:.3g} = {ratio:.3f} x tolerance"
+    again = gpu_decode(c, w)
+    assert np.array_equal(got, again)
+    assert c.read_device_status() == 0
