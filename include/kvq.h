@@ -139,8 +139,11 @@ size_t kvq_decode_workspace_bytes(const kvq_cache* cache, int32_t batch, int32_t
  *   out          [batch][n_q_heads][head_dim], fp32 if out_fp32 else bf16.
  *   softmax_scale  multiplier of q.k; 0 means 1/sqrt(head_dim).
  *   workspace    device scratch of >= kvq_decode_workspace_bytes(...) bytes,
- *                16-byte aligned, ZEROED BEFORE ITS FIRST USE; every call leaves
- *                it zeroed again.  Calls sharing a workspace must not overlap.
+ *                16-byte aligned, ZEROED BEFORE ITS FIRST USE: it holds the
+ *                partials of segments cut between CTAs and the merge counters,
+ *                which every call leaves zeroed again (the partials are
+ *                rewritten by each call).  Calls sharing a workspace must not
+ *                overlap.
  * For rotated K the kernel rotates q by the same Hadamard-256 (q.k is unchanged
  * because the rotation is orthonormal); for rotated V it rotates the output
  * back.  Page ids out of range are replaced by page 0 and recorded in the

@@ -2,7 +2,7 @@
 // memory.
 //
 // kvq_decode_attention needs a caller-provided device workspace for its split
-// partials and its grid-barrier word.  Some callers have no way to provide one: a
+// partials and its merge counters.  Some callers have no way to provide one: a
 // plugin handed only its input and output buffers by a host engine, a process
 // running under a fixed device-memory budget that forbids new allocations
 // after start-up, or a real-time loop where cudaMalloc/cudaFree (which may
