@@ -732,29 +732,41 @@ constexpr int kWsThreads = 512;
 constexpr int kDqWarps = 11;      // dequantising warps: 1..3 and 8..15
 constexpr int kWsBars = 15;       // kfull[2] vfull[2] kfree[2] sfull[2] sfree[2] pfull[2] pvdone[2] drain
 
+// 32 bytes from global memory (one 256-bit load; the address is 32-byte aligned)
+__device__ __forceinline__ void ldg256(const void* src, uint4& lo, uint4& hi) {
+    asm volatile("ld.global.nc.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(lo.x), "=r"(lo.y), "=r"(lo.z), "=r"(lo.w), "=r"(hi.x), "=r"(hi.y), "=r"(hi.z), "=r"(hi.w)
+                 : "l"(src));
+}
+
 // A dequantising thread's share of one key or value tile, read from the page
-// slab in global memory.  The tile's T x CPR 16-byte chunks are taken in
-// blocks of 8 rows x 4 chunks, one block per warp and step: lane l holds row
-// 8 rb + l % 8, chunk 4 cb + l / 8.  So a warp's loads cover 64 contiguous
-// bytes of each of 8 rows, and each 8-lane phase of its 16-byte shared-memory
-// stores writes one chunk column of 8 consecutive rows -- consecutive 16-byte
-// slots of the operand tile, free of bank conflicts.  Rows at or past `valid`
-// load as zero codes with zero scales, which dequantise to zeros.
+// slab in global memory.  A lane takes two adjacent 16-byte chunks of a row
+// (one 32-byte load; the row's chunk permutation XORs chunk indices with an
+// even value, or swaps the two of a pair for 16-bit codes, so a pair stays a
+// pair) and their scale bits (one load: the pair shares its INT8, E4M3-row or
+// MX group; E2M1's four scales are contiguous).  A warp's step covers RB rows
+// x 2 LR chunks, lane l holding row l % RB and the pair l / RB: each 8-lane
+// phase of its 16-byte shared-memory stores writes one chunk column of 8
+// consecutive rows -- consecutive 16-byte slots of the operand tile, free of
+// bank conflicts.  Rows at or past `valid` load as zero codes with zero
+// scales, which dequantise to zeros.
 template <int KIND, int D>
 struct DqShare {
     static constexpr int CB = row_code_bytes(KIND, D), SB = row_scale_bytes(KIND, D);
-    static constexpr int CPR = CB / 16;                // chunks per row: 4 .. 32
+    static constexpr int CPR = CB / 16;                     // chunks per row: 4 .. 32
+    static constexpr int LR = CPR / 2 < 4 ? CPR / 2 : 4;    // lanes per row in a step
+    static constexpr int RB = 32 / LR;                      // rows of a step: 8 or 16
     static constexpr int NW = kDqWarps;
-    static constexpr int NPT = ((kMaxT / 8) * (CPR / 4) + NW - 1) / NW;   // blocks per warp at T = 64
-    uint4 w[NPT > 0 ? NPT : 1];
-    uint32_t sb[NPT > 0 ? NPT : 1];
+    static constexpr int NPT = ((kMaxT / RB) * (CPR / (2 * LR)) + NW - 1) / NW;   // steps per warp at T = 64
+    uint4 w[NPT][2];
+    uint32_t sb[NPT];
 
-    // lgR = log2(T / 8): the tile's row blocks
-    __device__ __forceinline__ static void chunk_of(int i, int lgR, int dw, int l, int& t, int& j, bool& in) {
-        const int id = dw + i * NW;                    // block id
-        in = id < ((CPR / 4) << lgR);
-        t = ((id & ((1 << lgR) - 1)) << 3) + (l & 7);
-        j = ((id >> lgR) << 2) + (l >> 3);
+    // lgR = log2(T / RB): the tile's row blocks
+    __device__ __forceinline__ static void pair_of(int i, int lgR, int dw, int l, int& t, int& j, bool& in) {
+        const int id = dw + i * NW;                    // step id
+        in = id < ((CPR / (2 * LR)) << lgR);
+        t = (id & ((1 << lgR) - 1)) * RB + (l % RB);
+        j = (id >> lgR) * (2 * LR) + 2 * (l / RB);     // the pair's first chunk (even)
     }
     __device__ __forceinline__ void fetch(const uint8_t* codes, const uint8_t* scales, int r0, int lgR, int valid,
                                           int dw, int l) {
@@ -762,18 +774,22 @@ struct DqShare {
         for (int i = 0; i < NPT; i++) {
             int t, j;
             bool in;
-            chunk_of(i, lgR, dw, l, t, j, in);
-            w[i] = make_uint4(0, 0, 0, 0);
+            pair_of(i, lgR, dw, l, t, j, in);
+            w[i][0] = w[i][1] = make_uint4(0, 0, 0, 0);
             sb[i] = 0;
             if (in && t < valid) {
                 const int row = r0 + t;
-                w[i] = __ldg(reinterpret_cast<const uint4*>(codes + (int64_t)row * CB +
-                                                            ((j ^ row_swizzle(KIND, D, row)) << 4)));
+                const int pj = j ^ row_swizzle(KIND, D, row);   // physical chunk of j; j + 1 at pj ^ 1
+                uint4 lo, hi;
+                ldg256(codes + (int64_t)row * CB + ((pj & ~1) << 4), lo, hi);
+                w[i][0] = (pj & 1) ? hi : lo;
+                w[i][1] = (pj & 1) ? lo : hi;
                 if constexpr (SB > 0) {
                     const uint8_t* srow = scales + (int64_t)row * SB;
-                    if constexpr (kind_scale_bytes(KIND) == 2 || kind_bits(KIND) == 4) {
-                        const int off = kind_bits(KIND) == 4 ? 2 * j : 2 * (j * 16 / kind_group(KIND));
-                        sb[i] = __ldg(reinterpret_cast<const uint16_t*>(srow + off));
+                    if constexpr (kind_bits(KIND) == 4) {
+                        sb[i] = __ldg(reinterpret_cast<const uint32_t*>(srow + 2 * j));   // 2 chunks x 2 scales
+                    } else if constexpr (kind_scale_bytes(KIND) == 2) {
+                        sb[i] = __ldg(reinterpret_cast<const uint16_t*>(srow + 2 * (j * 16 / kind_group(KIND))));
                     } else {
                         sb[i] = __ldg(srow + j * 16 / kind_group(KIND));
                     }
@@ -786,8 +802,13 @@ struct DqShare {
         for (int i = 0; i < NPT; i++) {
             int t, j;
             bool in;
-            chunk_of(i, lgR, dw, l, t, j, in);
-            if (in) dequant_chunk<KIND, D>(w[i], sb[i], j, tile, t, T, smul);
+            pair_of(i, lgR, dw, l, t, j, in);
+            if (in) {
+                const uint32_t s1 = kind_bits(KIND) == 4 ? sb[i] >> 16 : sb[i];   // the second chunk's scale bits
+                dequant_chunk<KIND, D>(w[i][0], sb[i] & (kind_bits(KIND) == 4 ? 0xFFFFu : 0xFFFFFFFFu), j, tile, t, T,
+                                       smul);
+                dequant_chunk<KIND, D>(w[i][1], s1, j + 1, tile, t, T, smul);
+            }
         }
     }
 };
@@ -799,7 +820,7 @@ __global__ void __launch_bounds__(kWsThreads, 1) prefill_ws_kernel(const Prefill
     constexpr int OST = D + 4;
     constexpr uint32_t kCols = D == 256 ? 512 : 256;   // O in [0, D), S(b) in [D + 64 b, D + 64 b + 64)
     extern __shared__ __align__(1024) uint8_t smem[];
-    const int T = p.T, lgR = 28 - __clz(T);       // log2(T / 8)
+    const int T = p.T, lgT = 31 - __clz(T);
     uint8_t* sQ = smem;
     uint8_t* sK0 = sQ + kPrefillRows * D * 2;     // sK(b) = sK0 + b T D 2
     uint8_t* sV0 = sK0 + 2 * T * D * 2;
@@ -1016,6 +1037,8 @@ __global__ void __launch_bounds__(kWsThreads, 1) prefill_ws_kernel(const Prefill
             const int dw = warp < 4 ? warp - 1 : warp - 5;   // dequantising warp 0..10
             DqShare<KK, D> rk;
             DqShare<KV, D> rv;
+            // log2(T / RB) of each array's steps (T >= RB: tiles of 16 tokens or more)
+            const int lgRk = lgT - (DqShare<KK, D>::RB == 16 ? 4 : 3), lgRv = lgT - (DqShare<KV, D>::RB == 16 ? 4 : 3);
             // tile k + 1's codes are loaded while tile k is converted, and tile
             // k + 2's block-table entry with them, so no load waits on another
             int r0 = 0;
@@ -1023,13 +1046,13 @@ __global__ void __launch_bounds__(kWsThreads, 1) prefill_ws_kernel(const Prefill
             int pid_next = ntiles > 1 ? tile_pid(1) : 0;
             int valid = min(T, Ls);
             if (ntiles > 0) {
-                rk.fetch(slab, slab + p.L.off_ks, r0, lgR, valid, dw, lane);
-                rv.fetch(slab + p.L.off_vc, slab + p.L.off_vs, r0, lgR, valid, dw, lane);
+                rk.fetch(slab, slab + p.L.off_ks, r0, lgRk, valid, dw, lane);
+                rv.fetch(slab + p.L.off_vc, slab + p.L.off_vs, r0, lgRv, valid, dw, lane);
             }
             for (int k = 0; k < ntiles; k++) {
                 const uint32_t g = gk + k, bb = g & 1u, ph = (g >> 1) & 1u;
                 if (k >= 2 && !wait_warp(KFREE + bb, ph ^ 1u)) break;   // S of tile g - 2 done with sK(b)
-                rk.store(sK(bb), T, lgR, dw, lane, kmul);
+                rk.store(sK(bb), T, lgRk, dw, lane, kmul);
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(KFULL + bb));
@@ -1038,15 +1061,15 @@ __global__ void __launch_bounds__(kWsThreads, 1) prefill_ws_kernel(const Prefill
                 if (k + 1 < ntiles) {
                     slab1 = tile_slab(pid_next, k + 1, r1);
                     valid = min(T, Ls - (k + 1) * T);
-                    rk.fetch(slab1, slab1 + p.L.off_ks, r1, lgR, valid, dw, lane);
+                    rk.fetch(slab1, slab1 + p.L.off_ks, r1, lgRk, valid, dw, lane);
                     pid_next = k + 2 < ntiles ? tile_pid(k + 2) : 0;
                 }
                 if (k >= 2 && !wait_warp(PVDONE + bb, ph ^ 1u)) break;   // P V of tile g - 2 done with sV(b)
-                rv.store(sV(bb), T, lgR, dw, lane, vmul);
+                rv.store(sV(bb), T, lgRv, dw, lane, vmul);
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(VFULL + bb));
-                if (k + 1 < ntiles) rv.fetch(slab1 + p.L.off_vc, slab1 + p.L.off_vs, r1, lgR, valid, dw, lane);
+                if (k + 1 < ntiles) rv.fetch(slab1 + p.L.off_vc, slab1 + p.L.off_vs, r1, lgRv, valid, dw, lane);
             }
         }
         gk += (uint32_t)ntiles;
