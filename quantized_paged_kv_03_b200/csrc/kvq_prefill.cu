@@ -954,7 +954,9 @@ __global__ void __launch_bounds__(kWsThreads, 1) prefill_ws_kernel(const Prefill
             const int pos = gr < rows_total ? Ls - n + (int)(gr / p.G) : -1;
             const int64_t gfirst = R0 + g4 * 32;
             const int gpos_min = gfirst + 31 < rows_total ? Ls - n + (int)(gfirst / p.G) : -1;
-            const float qm = p.q_mult * pow2i(ek_seq) * qrm[r];
+            // this row's score multiplier, kept positive (masked scores are -inf
+            // and go through fma(s, qm, -base))
+            const float qm = fmaxf(p.q_mult * pow2i(ek_seq) * qrm[r], 1.17549435e-38f);
             float m_ref = -INFINITY;
             l_row = 0.f;
             bool ok = true;
@@ -974,17 +976,18 @@ __global__ void __launch_bounds__(kWsThreads, 1) prefill_ws_kernel(const Prefill
                 tc::fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(SFREE + bb));   // S(b) may be overwritten
+                // raw scores: the row's multiplier qm > 0 goes into the exponent
+                // (fma(s, qm, -base)), so the maximum is taken over the raw values
                 const int t0 = k * T;
-                const bool mask = t0 + T - 1 > gpos_min;
+                if (t0 + T - 1 > gpos_min || T < 64) {   // keys past the tile or past a row's position
+#pragma unroll
+                    for (int i = 0; i < 64; i++)
+                        if (i >= T || t0 + i > pos) v[i] = __float_as_uint(-INFINITY);
+                }
                 float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // four chains for latency
 #pragma unroll
-                for (int i = 0; i < 64; i++) {
-                    float x = __uint_as_float(v[i]) * qm;
-                    if (i >= T || (mask && t0 + i > pos)) x = -INFINITY;
-                    v[i] = __float_as_uint(x);
-                    mx4[i & 3] = fmaxf(mx4[i & 3], x);
-                }
-                const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+                for (int i = 0; i < 64; i++) mx4[i & 3] = fmaxf(mx4[i & 3], __uint_as_float(v[i]));
+                const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * qm;
                 float corr = 1.f;
                 const bool resc = mx > m_ref + 8.f;
                 if (resc) {
@@ -999,8 +1002,8 @@ __global__ void __launch_bounds__(kWsThreads, 1) prefill_ws_kernel(const Prefill
                     uint32_t hw[4];
 #pragma unroll
                     for (int i = 0; i < 4; i++) {
-                        const float pa = ex2(__uint_as_float(v[8 * q8 + 2 * i]) - base);
-                        const float pb = ex2(__uint_as_float(v[8 * q8 + 2 * i + 1]) - base);
+                        const float pa = ex2(fmaf(__uint_as_float(v[8 * q8 + 2 * i]), qm, -base));
+                        const float pb = ex2(fmaf(__uint_as_float(v[8 * q8 + 2 * i + 1]), qm, -base));
                         rs4[i] += pa + pb;
                         hw[i] = f16x2_of(pa, pb);
                     }
