@@ -778,7 +778,8 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
                 // multiple of 64, so the row's chunk permutation is the same.
                 const int t = (seq_len - 1) - span * U.sp;
                 const int tp = t + (span & ((1 << U.lg_up) - 1)) * U.sp;
-                const int role = wpu >= 2 ? tile : 2;   // 0: K row, 1: V row, 2: both
+                // 0: K row, 1: V row, 2: both (a group of one warp), 3: neither
+                const int role = wpu >= 2 ? (tile < 2 ? tile : 3) : 2;
                 if (role <= 2) {
                     uint8_t* g = (hb == 0) ? p.slabs + (int64_t)(unit_src(u) >> 2) * slab : nullptr;
                     const int64_t row = (int64_t)b * H + h;
