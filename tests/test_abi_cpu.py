@@ -66,6 +66,31 @@ def test_cache_bytes_is_header_plus_slabs(L):
         assert n == 256 + 2 * 5 * 3 * P * K.token_bytes(fmt, D), fmt
 
 
+def test_slab_regions_are_32_byte_aligned(L):
+    """The prefill kernel reads a row's 16-byte code chunks in pairs with one
+    32-byte load, and the pool starts 256-byte aligned: every code row, every
+    region of a page slab (K codes, K scales, V codes, V scales) and the slab
+    itself must then be whole multiples of 32 bytes, for every format, head_dim
+    and page size the cache accepts.  The slab size is read back from the pool
+    size (header + layers x pages x heads x slab)."""
+    a16 = lambda x: (x + 15) // 16 * 16
+    checked = 0
+    for fmt in sorted(K.FORMATS):
+        for D in (128, 256):
+            if K.token_bytes(fmt, D) == 0:
+                continue
+            kc, ks = K.row_bytes(fmt, D, False)
+            vc, vs = K.row_bytes(fmt, D, True)
+            assert kc % 32 == 0 and vc % 32 == 0, (fmt, D)
+            for P in range(16, 257, 16):
+                regions = [a16(P * kc), a16(P * ks), a16(P * vc), a16(P * vs)]
+                assert all(r % 32 == 0 for r in regions), (fmt, D, P, regions)
+                slab = K.cache_bytes(fmt, D, n_kv_heads=1, page_size=P, num_pages=1, flags=K.FLAG_NO_ROTATE) - 256
+                assert slab == sum(regions) and slab % 32 == 0, (fmt, D, P, slab)
+                checked += 1
+    assert checked >= 12 * 16
+
+
 def _desc(**kw):
     base = dict(fmt=K.FORMATS["int8_g64"], D=256, H=2, P=64, pages=4, layers=1, flags=0)
     base.update(kw)
