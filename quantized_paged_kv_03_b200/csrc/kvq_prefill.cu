@@ -1165,8 +1165,11 @@ static constexpr size_t kSmemLimit = 227 * 1024;   // opt-in shared memory per C
 cudaError_t plan_prefill(const Layout& L, PrefillPlan* plan) {
     int T = 64;
     while (L.P % T) T >>= 1;   // the largest of 64, 32, 16 that divides the page
-    {
-        // the warp-specialised kernel, whenever its tiles fit
+    // the warp-specialised kernel, whenever its tiles fit and the slab's rows
+    // and regions allow its 32-byte loads (true of every layout today)
+    const bool a32 = L.kc % 32 == 0 && L.vc % 32 == 0 && L.off_ks % 32 == 0 && L.off_vc % 32 == 0 &&
+                     L.off_vs % 32 == 0 && L.slab % 32 == 0;
+    if (a32) {
         PrefillPlan q;
         memset(&q, 0, sizeof(q));
         q.T = T;
