@@ -59,8 +59,8 @@ KERNEL_SOURCES = ("kvq_decode.cu", "kvq_common.cuh", "kvq_quant.cuh", "kvq_inter
 
 
 # The same for the chunked-prefill kernel on its workload.
-PREFILL_TRAFFIC = {"bytes": 173_243_029 + 38_804_971,
-                   "sources_sha256": "abb7c0f726750e66e114193f24c5f9841ff7f946fc64aa00a01c37ea1923b3c9"}
+PREFILL_TRAFFIC = {"bytes": 173_958_912 + 38_617_515,
+                   "sources_sha256": "317fa9a46181eca3319643d4c7bc3ffde291a7a013326c6d7185427ff47037b8"}
 PREFILL_SOURCES = ("kvq_prefill.cu", "kvq_prefill.h", "kvq_tc.cuh", "kvq_common.cuh")
 
 
