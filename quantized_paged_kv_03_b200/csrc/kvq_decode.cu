@@ -47,6 +47,13 @@ constexpr int kDecThreads = 256;   // 8 warps, each a 16-token tile over all of 
 template <int D>
 constexpr int kOsmStride = D + 4;
 constexpr int kMaxStages = 8;
+// A segment's fused append is quantised at the segment start when the range
+// holds at most this many of its units (its last unit then comes within about
+// the ring's first fill), else when its last unit's data have arrived.  Only
+// for INT8-G64 (fused_early): there it shortened the step by 6 %, while on the
+// other formats the extra path cost the unit loop 1-2 % whether it ran or not.
+constexpr int kFusedEarly = 16;
+__host__ __device__ constexpr bool fused_early(int kk, int kv) { return kk == RK_INT8_G64 && kv == RK_INT8_G64; }
 constexpr int kMaxBatch = 4096;
 // Parts of a cut segment merged together by the CTA that completes them: a
 // segment of more parts is merged in groups of this many, then the groups.
@@ -424,6 +431,32 @@ __device__ __noinline__ void fused_append_rows(int role, int lane, const uint16_
     }
 }
 
+// The same rows quantised ahead of their unit (which == 0: K, 1: V) into a
+// row buffer -- K codes at 0, K scales at KC, V codes at KC + 16, V scales at
+// KC + 16 + VC (FusedRow) -- in row t's chunk permutation, and, when g is set,
+// into the cache slab.
+template <int KK, int KV, int D>
+struct FusedRow {
+    using T = DecTraits<KK, KV, D>;
+    static constexpr int ks = T::KC, vc = T::KC + 16, vs = T::KC + 16 + T::VC;
+    static_assert(T::KS <= 16 && T::VS <= 16 && T::KC % 16 == 0 && T::VC % 16 == 0, "row buffer layout");
+    static_assert(T::KC <= 512 && T::VC <= 512, "one 16-byte piece per lane");
+};
+template <int KK, int KV, int D>
+__device__ __noinline__ void fused_append_buf(int which, int lane, const uint16_t* src, bool rot, float tscale,
+                                              uint8_t* buf, uint8_t* g, int t, int tp, int c_ks, int c_vc,
+                                              int c_vs) {
+    using T = DecTraits<KK, KV, D>;
+    using R = FusedRow<KK, KV, D>;
+    if (which == 0) {
+        quantize_row<KK, D>(src, rot, tscale, buf, buf + R::ks, t, lane, g ? g + tp * T::KC : nullptr,
+                            g ? g + c_ks + tp * T::KS : nullptr);
+    } else {
+        quantize_row<KV, D>(src, rot, tscale, buf + R::vc, buf + R::vs, t, lane,
+                            g ? g + c_vc + tp * T::VC : nullptr, g ? g + c_vs + tp * T::VS : nullptr);
+    }
+}
+
 template <int KK, int KV, int D, bool FUSED>
 __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_kernel(const DecodeParams p) {
     using T = DecTraits<KK, KV, D>;
@@ -738,6 +771,25 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
                     reinterpret_cast<uint2*>(qst)[slot] = make_uint2(pack_f16(v[0], v[1]), pack_f16(v[2], v[3]));
                 }
             }
+            if (FUSED && fused_early(KK, KV) && warp >= 6 && span0 + seg_n == nspans && seg_n <= kFusedEarly) {
+                // fused append ahead of its unit: the range reaches the segment's
+                // last unit soon, so its copies are in flight now.  Warp 6
+                // quantises the newest token's K row, warp 7 its V row, into the
+                // row buffer in the output-combine area (untouched until the
+                // segment's units are done) and, for head block 0, into the cache.
+                const int span = nspans - 1;
+                const int t = (seq_len - 1) - span * U.sp;
+                if (t < U.sp) {
+                    const int tp = t + (span & ((1 << U.lg_up) - 1)) * U.sp;
+                    uint8_t* g = (hb == 0) ? p.slabs + (int64_t)(unit_src(i + seg_n - 1) >> 2) * slab : nullptr;
+                    const int64_t row = ((int64_t)b * H + h) * D;
+                    const int which = warp - 6;
+                    fused_append_buf<KK, KV, D>(which, lane, (which ? p.v_new : p.k_new) + row,
+                                                which ? p.rot_v : p.rot_k, which ? p.v_scale : p.k_scale,
+                                                reinterpret_cast<uint8_t*>(osm), g, t, tp, (int)p.L.off_ks,
+                                                (int)p.L.off_vc, (int)p.L.off_vs);
+                }
+            }
         }
         __syncthreads();
         hm0 = qhm[2 * j];
@@ -776,10 +828,30 @@ __global__ void __launch_bounds__(kDecThreads, decode_ctas(KK, KV, D)) decode_ke
                 // over whatever the copy brought, and into the cache (row tp of the
                 // page; one head block writes the cache).  t and tp differ by a
                 // multiple of 64, so the row's chunk permutation is the same.
+                // A sequence longer than its block table (flagged by the unit
+                // prefix) has no row to append: t would fall outside the unit.
+                // With few of the segment's units in the range the row was
+                // quantised at the segment start; the warp that owns row t's tile
+                // (the only one that reads it) copies it from the row buffer.
                 const int t = (seq_len - 1) - span * U.sp;
                 const int tp = t + (span & ((1 << U.lg_up) - 1)) * U.sp;
                 // 0: K row, 1: V row, 2: both (a group of one warp), 3: neither
-                const int role = wpu >= 2 ? (tile < 2 ? tile : 3) : 2;
+                const int role = t >= U.sp                                 ? 3
+                                 : fused_early(KK, KV) && seg_n <= kFusedEarly ? 4
+                                 : wpu >= 2                                    ? (tile < 2 ? tile : 3)
+                                                                               : 2;
+                if (role == 4 && tile == (t >> 4) % wpu) {
+                    using R = FusedRow<KK, KV, D>;
+                    const uint8_t* fb = reinterpret_cast<const uint8_t*>(osm);
+                    uint8_t* st = smem + stg;
+                    if (lane < T::KC / 16)
+                        reinterpret_cast<uint4*>(st + t * T::KC)[lane] = reinterpret_cast<const uint4*>(fb)[lane];
+                    if (lane < T::VC / 16)
+                        reinterpret_cast<uint4*>(st + off_vc + t * T::VC)[lane] =
+                            reinterpret_cast<const uint4*>(fb + R::vc)[lane];
+                    if (lane < T::KS) st[off_ks + t * T::KS + lane] = fb[R::ks + lane];
+                    if (lane < T::VS) st[off_vs + t * T::VS + lane] = fb[R::vs + lane];
+                }
                 if (role <= 2) {
                     uint8_t* g = (hb == 0) ? p.slabs + (int64_t)(unit_src(u) >> 2) * slab : nullptr;
                     const int64_t row = (int64_t)b * H + h;
