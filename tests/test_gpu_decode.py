@@ -134,7 +134,11 @@ def test_decode_many_sequences_balanced_split():
     ("mxfp8_g32", 4, 128, 128, [600, 128, 1], 2, 16),
     ("fp8_tensor", 4, 128, 64, [512, 77], 2, 16),
     ("bf16", 4, 128, 64, [300, 2], 2, 16),
-    ("int8_g64", 1, 256, 256, [700, 193, 64], 1, 8)])
+    ("int8_g64", 1, 256, 256, [700, 193, 64], 1, 8),
+    # one 330 000-token sequence on one kv-head: every CTA's range holds about
+    # 17 of the segment's units, so the new token is quantised when its unit
+    # arrives rather than at the segment start (the INT8 kernel's other path)
+    pytest.param("int8_g64", 1, 256, 64, [330000], 1, 4, id="int8_g64-long_ranges")])
 def test_fused_append_decode_equals_append_then_decode(fmt, cfg, D, P, lengths, H, Hq):
     """kvq_append_decode stores the same codes as kvq_append and returns the
     same output as kvq_decode_attention run after it."""
