@@ -34,6 +34,13 @@
  *       [-127, 127], byte = exponent + 127; amax = 0 gives byte 0 and +0 codes.
  *   R9  K8V4: K is FP8-E4M3 row-256 (not rotated), V is NVFP4-G16 rotated.
  *  R10  BF16 format: K is the bf16 bit pattern, V is fp16 (RNE, saturating).
+ *
+ * Parity unpinned: every function below is pinned by value (tests/
+ * test_oracle_pins.py: closed forms, brute force over the format grids,
+ * library routines), but the bit-level choices of R1 (butterfly order), R2
+ * (rounding direction of a scale), R3 (zero scale) and R7 (nibble order) are
+ * readings no page fixes; the CUDA path agrees with them because it follows
+ * the same readings, not because the pages confirm them.
  */
 #include <math.h>
 #include <stdint.h>
