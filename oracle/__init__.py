@@ -79,6 +79,7 @@ def lib():
             "or_quantize_rows": (i32, [i32, i32, ctypes.c_uint, f32, i32, i64, P, P, P]),
             "or_dequant_rows": (i32, [i32, i32, f32, i32, i64, P, P, P]),
             "or_attend": (i32, [i32, i64, i32, P, i32, i32, P, P, f64, P]),
+            "or_mla_attend": (i32, [i32, i32, i64, i32, P, P, f64, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -243,6 +244,22 @@ def attend(q: np.ndarray, k: np.ndarray, v: np.ndarray, k_rot: bool, v_rot: bool
     return out
 
 
+def mla_attend(q: np.ndarray, kv: np.ndarray, DC: int, scale: float) -> np.ndarray:
+    """fp64 MLA latent attention (absorbed form) of G query rows q [G, DC + DR]
+    over L cached rows kv [L, DC + DR]: scores from the latent and rotary parts,
+    values = the latent part.  Returns [G, DC]."""
+    q = np.ascontiguousarray(q, dtype=np.float64)
+    kv = np.ascontiguousarray(kv, dtype=np.float64)
+    G, W = q.shape
+    L = kv.shape[0]
+    if kv.shape[1] != W or not 0 < DC <= W:
+        raise ValueError("oracle mla_attend: row widths differ")
+    out = np.empty((G, DC), np.float64)
+    if lib().or_mla_attend(DC, W - DC, L, G, _ptr(q), _ptr(kv), float(scale), _ptr(out)) != 0:
+        raise ValueError("oracle mla_attend: invalid sizes")
+    return out
+
+
 def bf16_bits_to_f64(x: np.ndarray) -> np.ndarray:
     return (np.asarray(x, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
@@ -374,3 +391,62 @@ class PagedCache:
 def kv_elements(B: int, L: int, H_kv: int, S: int, d_head: int) -> int:
     """[llama.cpp] M_KV = 2 x B x L x H_kv x S x d_head (elements, K and V)."""
     return 2 * B * L * H_kv * S * d_head
+
+
+# ------------------------------------------------------ MLA latent cache
+
+class MLAPagedCache:
+    """Paged store of an MLA latent cache: one row of DC + DR values per token
+    (latent, then rotary key), no kv-head dimension -- every query head reads
+    the same row.  Stored as BF16 (the row's bits) or as FP8-E4M3 with one
+    per-tensor scale over the whole row ([TokenSpeed] fp8 KV switch, used with
+    its trtllm_mla backend).  Widths and the absorbed form: DeepSeek-V2 report,
+    "Multi-Head Latent Attention" (DC = 512, DR = 64); pages of page_size
+    tokens as in [NInfer]'s paging remark."""
+
+    def __init__(self, fmt: int, num_pages: int, page_size: int = 64, DC: int = 512, DR: int = 64,
+                 tensor_scale: float = 1.0):
+        if fmt not in (BF16, FP8_TENSOR):
+            raise ValueError("MLA latent cache: BF16 or FP8 per-tensor only")
+        self.fmt, self.P, self.num_pages, self.DC, self.DR = fmt, page_size, num_pages, DC, DR
+        self.scale = tensor_scale
+        cb, _ = row_bytes(fmt, False, DC + DR)
+        self.codes = np.zeros((num_pages * page_size, cb), np.uint8)
+
+    def row_bytes(self) -> int:
+        return self.codes.shape[1]
+
+    def append(self, rows_bf16: np.ndarray, slot_mapping: np.ndarray):
+        """Write latent rows [T, DC + DR] (bf16 bits) at slots; a negative slot skips."""
+        slots = np.asarray(slot_mapping, np.int64)
+        keep = slots >= 0
+        if not keep.any():
+            return
+        x = np.ascontiguousarray(rows_bf16[keep], np.uint16)
+        codes, _ = quantize_rows(self.fmt, False, x[:, None, :], 0, self.scale)
+        self.codes[slots[keep]] = codes.reshape(len(x), -1)
+
+    def dequant(self, slots: np.ndarray) -> np.ndarray:
+        empty = np.zeros((len(slots), 0), np.uint8)
+        return dequant_rows(self.fmt, False, np.ascontiguousarray(self.codes[slots]), empty,
+                            self.DC + self.DR, self.scale)
+
+    def decode(self, q_bf16: np.ndarray, block_table: np.ndarray, seq_lens: np.ndarray,
+               scale: float) -> np.ndarray:
+        """q [B, Hq, DC + DR] bf16 bits (absorbed latent query, then rotary
+        query) -> latent outputs [B, Hq, DC] fp64; a zero-length sequence
+        gives zero rows.  `scale` is the model's softmax scale (for the
+        DeepSeek-V2 shape 1/sqrt(128 + 64), the width of a head's un-absorbed
+        query), not 1/sqrt(DC + DR)."""
+        B, Hq, W = q_bf16.shape
+        if W != self.DC + self.DR:
+            raise ValueError("MLA decode: query width differs from the cache rows")
+        out = np.zeros((B, Hq, self.DC), np.float64)
+        for b in range(B):
+            n = int(seq_lens[b])
+            if n <= 0:
+                continue
+            t = np.arange(n)
+            slots = np.asarray(block_table[b], np.int64)[t // self.P] * self.P + t % self.P
+            out[b] = mla_attend(bf16_bits_to_f64(q_bf16[b]), self.dequant(slots), self.DC, scale)
+        return out

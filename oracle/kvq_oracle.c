@@ -34,6 +34,12 @@
  *       [-127, 127], byte = exponent + 127; amax = 0 gives byte 0 and +0 codes.
  *   R9  K8V4: K is FP8-E4M3 row-256 (not rotated), V is NVFP4-G16 rotated.
  *  R10  BF16 format: K is the bf16 bit pattern, V is fp16 (RNE, saturating).
+ *  R11  MLA latent cache (or_mla_attend): one row of DC + DR values per token
+ *       (DeepSeek-V2 report: DC = 512 latent, DR = 64 rotary key), shared by
+ *       every query head, attended in the absorbed form; the value is the
+ *       latent part of the same row.  FP8 storage is the per-tensor format of
+ *       [TokenSpeed]'s fp8 switch applied to the whole row (576 B per token
+ *       against 1152 B in BF16: the table's 0.5x).
  *
  * Parity unpinned: every function below is pinned by value (tests/
  * test_oracle_pins.py: closed forms, brute force over the format grids,
@@ -491,6 +497,55 @@ int or_attend(int D, int64_t L, int G, const double* q, int k_rot, int v_rot,
                 og[i] = acc[i];
             }
         }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------ MLA latent decode */
+
+/* Decode attention over a multi-head latent attention (MLA) cache, in fp64,
+ * absorbed form.  [TokenSpeed] recipe section (Kimi K2.5 served with
+ * --attention-backend trtllm_mla and --kv-cache-dtype fp8) and the GLM 8xB200
+ * deployment page (DSA+MLA) name the method; its shape comes from the
+ * DeepSeek-V2 report, section "Multi-Head Latent Attention" (R11).
+ * One cached row per token serves every query head: DC latent values c_t
+ * (the compressed key-value, which is also the value) followed by DR values
+ * r_t (the decoupled rotary key, shared by the heads).  A head's query row is
+ * (q_lat, q_rope), q_lat = W_UK^T q_nope already carrying the key
+ * up-projection, so that q_lat . c_t = q_nope . (W_UK c_t):
+ *   s_t = scale * (q_lat . c_t + q_rope . r_t);  p = softmax(s);
+ *   o = sum_t p_t c_t   (the latent output; W_UV is applied after attention).
+ * q: [G][DC + DR]; kv: [L][DC + DR]; out: [G][DC].  Returns -1 on bad sizes. */
+int or_mla_attend(int DC, int DR, int64_t L, int G, const double* q, const double* kv,
+                  double scale, double* out)
+{
+    if (L <= 0 || DC <= 0 || DR < 0 || DC + DR > 4096 || G <= 0) return -1;
+    const int W = DC + DR;
+    double acc[4096];
+    for (int g = 0; g < G; g++) {
+        const double* qg = q + (int64_t)g * W;
+        double m = -INFINITY;
+        for (int64_t t = 0; t < L; t++) {
+            const double* row = kv + t * W;
+            double lat = 0.0, rope = 0.0;
+            for (int i = 0; i < DC; i++) lat += qg[i] * row[i];
+            for (int i = 0; i < DR; i++) rope += qg[DC + i] * row[DC + i];
+            double s = scale * (lat + rope);
+            if (s > m) m = s;
+        }
+        double l = 0.0;
+        for (int i = 0; i < DC; i++) acc[i] = 0.0;
+        for (int64_t t = 0; t < L; t++) {
+            const double* row = kv + t * W;
+            double lat = 0.0, rope = 0.0;
+            for (int i = 0; i < DC; i++) lat += qg[i] * row[i];
+            for (int i = 0; i < DR; i++) rope += qg[DC + i] * row[DC + i];
+            double p = exp(scale * (lat + rope) - m);
+            l += p;
+            for (int i = 0; i < DC; i++) acc[i] += p * row[i];
+        }
+        double* og = out + (int64_t)g * DC;
+        for (int i = 0; i < DC; i++) og[i] = acc[i] / l;
     }
     return 0;
 }

@@ -262,6 +262,59 @@ def prefill_queries(w: Workload, q_lens, seed: int | None = None):
     return q, cu
 
 
+@dataclass
+class MLAWorkload:
+    """An MLA latent-cache decode case: one cached row of DC + DR values per
+    token (no kv-head dimension), Hq query rows per sequence."""
+    seed: int
+    B: int
+    Hq: int
+    DC: int
+    DR: int
+    P: int
+    seq_lens: np.ndarray      # int32 [B]
+    block_table: np.ndarray   # int32 [B, max_pages], -1 past each sequence
+    num_pages: int
+    rows: np.ndarray          # bf16 bits [T, DC + DR], sequences back to back
+    q: np.ndarray             # bf16 bits [B, Hq, DC + DR]
+    starts: np.ndarray        # int64 [B + 1] first row of each sequence
+
+    def slots(self) -> np.ndarray:
+        """Cache slot of every row (page of the block table x P + offset)."""
+        out = np.empty(int(self.starts[-1]), np.int64)
+        for b in range(self.B):
+            t = np.arange(int(self.seq_lens[b]))
+            out[self.starts[b]:self.starts[b + 1]] = self.block_table[b, t // self.P].astype(np.int64) * self.P + t % self.P
+        return out
+
+
+def make_mla_workload(seq_lens, Hq: int, seed: int, DC: int = 512, DR: int = 64, P: int = 64,
+                      outlier_frac: float = 0.02, outlier_gain: float = 20.0) -> MLAWorkload:
+    """Seeded MLA latent rows and queries: standard normals rounded to bf16,
+    with round(outlier_frac * (DC + DR)) outlier channels scaled by
+    outlier_gain (the same channels for every token); the queries N(0, 1).
+    Block tables as in make_workload: slices of one random page permutation."""
+    seq_lens = np.asarray(seq_lens, np.int32)
+    B, W = len(seq_lens), DC + DR
+    pages = [(int(L) + P - 1) // P for L in seq_lens]
+    num_pages = max(1, sum(pages))
+    perm = _rng(seed, 3).permutation(num_pages).astype(np.int32)
+    bt = np.full((B, max(1, max(pages) if pages else 1)), -1, np.int32)
+    o = 0
+    for b, n in enumerate(pages):
+        bt[b, :n] = perm[o:o + n]
+        o += n
+    starts = np.zeros(B + 1, np.int64)
+    starts[1:] = np.cumsum(seq_lens)
+    gain = np.ones(W, np.float32)
+    n_out = int(round(outlier_frac * W))
+    if n_out:
+        gain[_rng(seed, 7).choice(W, n_out, replace=False)] = outlier_gain
+    x = _rng(seed, 8).standard_normal((int(starts[-1]), W), dtype=np.float32) * gain
+    q = _rng(seed, 9).standard_normal((B, Hq, W), dtype=np.float32)
+    return MLAWorkload(seed, B, Hq, DC, DR, P, seq_lens, bt, num_pages, bf16_bits(x), bf16_bits(q), starts)
+
+
 def tensor_amax(x_bf16: np.ndarray) -> float:
     """Largest magnitude of a bf16 tensor (input statistic for a static scale)."""
     if x_bf16.size == 0:
